@@ -1,0 +1,317 @@
+"""Benchmark of the W4A4 ConvRot linear layer on B200.
+
+Workload (default): the Flux-like attention projection, M = 4608 tokens (4096
+image + 512 text), K = N = 3072, ConvRot group 128, bias, no low-rank branch.
+One step = one whole layer over one batch: rotate + quantize the bf16
+activations (K1), then the INT4 GEMM with the fused dequant + bias epilogue
+(K2) -- the same two launches w4a4_linear makes.  Inputs are synthetic
+(seeded NumPy draws in the shape and value mix of the pages' workload) and
+resident in HBM; four input sets (about 272 MB) rotate so that no step finds
+its inputs in the 126 MB L2.
+
+Prints one JSON line (rank 0).  Metric: TOPS = 2 M N K / time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one independent layer per GPU (weak scaling: the path shards by
+tokens with no exchange), timed on the device, max over ranks.
+--impl reference times the CPU oracle on the host cores on a bounded sample
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+INT8_NOMINAL_TOPS = 4500.0     # B200 dense INT8 tensor peak (datasheet)
+HBM_NOMINAL_GBS = 8000.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_init(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return rank, world, local
+
+
+def cpu_baseline(spec, budget_s: float = 10.0) -> dict:
+    """The CPU oracle as it stands, on the host cores, on a bounded sample of
+    the workload: the per-step path (activation rotate + quantize, integer
+    GEMM, epilogue) for a subset of token rows against the full weight matrix
+    (weights are quantized once, offline, as on the GPU)."""
+    import oracle
+    from w4a4_int4_quantized_b200 import inputs
+    d = inputs.make_layer(spec)
+    _, ws, wq = oracle.quantize_w4(d["W"], spec.group)
+    rows = 8
+    while True:
+        t0 = time.perf_counter()
+        _, xs, xq = oracle.quantize_w4(d["X"][:rows], spec.group)
+        acc = oracle.int_gemm(xq, wq)
+        oracle.epilogue(acc, xs, ws, spec.group, None, None, d["bias"])
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or rows >= spec.M:
+            break
+        rows = min(spec.M, max(rows * 2, int(rows * budget_s / max(dt, 1e-3) * 1.1)))
+    ops = 2.0 * rows * spec.N * spec.K
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows} of {spec.M} token rows x full {spec.N}x{spec.K} weights "
+                      f"(act quant + int GEMM + epilogue), {dt:.1f} s"}
+
+
+def run_reference(args, spec):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(spec, budget_s=budget / 4)
+    vals = [cpu_baseline(spec, budget_s=budget) for _ in range(args.steps)]
+    v = statistics.median([b["value"] for b in vals])
+    line = {
+        "impl": "reference", "metric": "W4A4 linear TOPS (M=4608, K=N=3072)", "value": v, "unit": "TOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 2.0 * spec.M * spec.N * spec.K / (v * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes, int64 acc, f64 epilogue",
+        "data": "synthetic", "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N,
+                                        "group": spec.group, "rank": spec.rank},
+        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": vals[0]["cores"], "kind": "oracle",
+                         "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="attn_proj")
+    ap.add_argument("--sets", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    from w4a4_int4_quantized_b200 import inputs
+    spec = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, spec)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import w4a4_int4_quantized_b200 as w4
+
+    rank, world, local = _dist_init(args.gpus)
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w4.load_library()
+    g, M, K, N, r = spec.group, spec.M, spec.K, spec.N, spec.rank
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    sets = []
+    for i in range(args.sets):
+        d = inputs.make_layer(spec, seed_offset=1000 * rank + i)
+        X = dev(d["X"])
+        Wq, ws = w4.w4a4_quantize_weights(dev(d["W"]), g)
+        s = dict(X=X, Wq=Wq, ws=ws, bias=dev(d["bias"]) if d["bias"] is not None else None,
+                 L1=dev(d["L1"]) if r else None, L2=dev(d["L2"]) if r else None,
+                 Xq=torch.empty((M, K // 2), dtype=torch.uint8, device="cuda"),
+                 xs=torch.empty((M,), dtype=torch.float32, device="cuda"),
+                 T=torch.empty((M, r), dtype=torch.bfloat16, device="cuda") if r else None,
+                 Y=torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
+        sets.append(s)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(s, ev=None):
+        w4.w4a4_rotate_quantize_act(s["X"], g, s["L1"], Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=stream)
+        if ev is not None:
+            ev.record(stream)
+        w4.w4a4_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], g, s["T"], s["L2"], s["bias"], Y=s["Y"], stream=stream)
+
+    for i in range(args.warmup):
+        step(sets[i % len(sets)])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(sets[i % len(sets)], ev[i][1])
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    k1_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    k2_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    err = w4.w4a4_get_device_error()
+    if err:
+        raise SystemExit(f"device error word {err:#x}")
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ops = 2.0 * M * N * K
+    value = ops * args.steps * world / (total_ms * 1e-3) / 1e12
+
+    # end to end through the public call: pinned host X in, host Y out
+    e2e = None
+    if args.e2e_steps > 0:
+        s = sets[0]
+        hx = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+        hx.copy_(s["X"].cpu())
+        hy = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+        ws_buf = torch.empty((w4.w4a4_workspace_bytes(M, K, r),), dtype=torch.uint8, device="cuda")
+        for _ in range(3):
+            s["X"].copy_(hx, non_blocking=True)
+            w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"], workspace=ws_buf)
+            hy.copy_(s["Y"], non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            s["X"].copy_(hx, non_blocking=True)
+            w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"], workspace=ws_buf)
+            hy.copy_(s["Y"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": ops * args.e2e_steps * world / (float(te.item()) * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2}
+
+    if rank == 0:
+        pk = _peaks()
+        k1 = statistics.mean(k1_ms)
+        k2 = statistics.mean(k2_ms)
+        k2_tops = ops / (k2 * 1e-3) / 1e12
+        int8_peak = 2.0 * pk["bf16_sustained"]   # nominal int8 : bf16 ratio is 2
+        k1_bytes = M * K * 2 + M * K // 2 + M * 4
+        line = {
+            "metric": "W4A4 linear TOPS & us/layer (M=4608,K=N=3072) and % of B200 INT8 TC peak",
+            "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "us_per_layer": total_ms / args.steps * 1e3,
+            "frac_of_int8_nominal_peak": value / INT8_NOMINAL_TOPS,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int4 codes (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
+            "config": {"workload": spec.name, "M": M, "K": K, "N": N, "group": g, "rank": r,
+                       "bias": spec.bias, "parallelism": f"replicas x{world} (token shards, no exchange)",
+                       "l2": f"{args.sets} rotating input sets (> L2)"},
+            "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3},
+            "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
+                         "frac": k2_tops / int8_peak, "traffic": None,
+                         "peak_note": f"int8 = 2 x {pk['source']} sustained bf16 {pk['bf16_sustained']} TFLOP/s"},
+            "roofline_k1": {"bound": "hbm", "achieved": k1_bytes / (k1 * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                            "unit": "GB/s", "frac": k1_bytes / (k1 * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "gpu_launches": 2 * args.steps + (args.steps if r else 0),
+            "clocks": clk, "wall_s": wall, "e2e": e2e,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(spec)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

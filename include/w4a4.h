@@ -1,0 +1,171 @@
+/*
+ * libw4a4 -- W4A4 ConvRot INT4 linear layer (and its W8A8 twin) for NVIDIA
+ * B200 (sm_100a).  C ABI: plain pointers, sizes and a CUDA stream.
+ *
+ * The method, in the words of the pages it comes from (restated):
+ *   - "Load Diffusion Model INT4 (W4A4)" (comfy.icu), intro: every layer is
+ *     quantized to 4-bit weights and 4-bit activations, with a Hadamard
+ *     rotation (ConvRot) applied first so that the quantization error does not
+ *     concentrate in outlier channels; the matmuls then run on integer tensor
+ *     cores.  "The inputs you'll actually touch": enable_convrot (on by
+ *     default), groupsize, on-the-fly quantization from BF16/FP16 only.
+ *   - "W4A4 and W4A8: The New Quantization Toolkit" (renderbob.io), "Decoding
+ *     the notation": weights are quantized once, activations on the fly;
+ *     "How the toolkit tells you to choose": W8A8 covers layers that do not
+ *     tolerate 4 bit, and a caller falls back to it on incompatible shapes.
+ *   - "Krea 2 Turbo - SVDQuant" (sweettea.co), "What's included": an optional
+ *     low-rank branch (X L1) L2 corrects the quantized product.
+ *   - "Save Int4 Model" (comfy.icu), "How it works": one weight_scale per
+ *     quantized tensor, a convrot group size recorded per layer.
+ *
+ * Arithmetic (readings of the pages, identical in the CPU oracle):
+ *   H_g[i][j] = (-1)^popcount(i & j), g in {64, 128}; group 0 = no rotation.
+ *   Rotation: each group of g consecutive entries along K is multiplied by the
+ *     unnormalised H_g in fp32 (butterflies in the order h = 1, 2, 4, ...).
+ *   Scale: s = fl32(max_k |y_k| / qmax), one per row (token or output channel);
+ *     qmax = 7 (INT4) or 127 (INT8); s = 0 for an all-zero row.
+ *   Codes: q = rint_half_even(fl32(y / s)) (IEEE division), |q| <= qmax.
+ *   INT4 packing: row-major [rows, K/2] bytes; byte j holds code 2j in bits
+ *     0..3 and code 2j+1 in bits 4..7, 4-bit two's complement.
+ *   GEMM: acc[m][n] = sum_k qx[m][k] * qw[n][k], exact int32.
+ *   Epilogue: Y = bf16_rn( ((acc * s_x[m]) * s_w[n]) * (1/g)
+ *                          + sum_j T[m][j] L2[j][n] + bias[n] ),
+ *     T = X L1 from the unrotated activations (fp32 sums, stored as bf16).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are caller-owned CUDA device memory, row-major and contiguous,
+ *     with 16-byte-aligned base addresses (32-byte for the code tensors Xq and
+ *     Wq given to the GEMMs).  bf16 tensors are passed as void*.
+ *     The library never allocates on these paths and keeps no state besides
+ *     per-device launch attributes and the device error word.
+ *   - Calls are asynchronous and ordered on `stream` (NULL = legacy default
+ *     stream).  W4A4_OK means "validated and enqueued"; launch failures return
+ *     W4A4_ERR_CUDA; faults inside a kernel surface at the caller's next
+ *     synchronisation.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check launches nothing and returns the status named below.
+ *   - Shape rules: M >= 1; K a multiple of 128 with K / max(g, 128) <= 256
+ *     (K <= 32768; K <= 16384 for g = 64); N a multiple of 8 (GEMM and linear);
+ *     group in {0, 64, 128}; rank r in [0, 256] and a multiple of 16.
+ *   - Only sm_100 devices are supported (W4A4_ERR_UNSUPPORTED_DEVICE
+ *     otherwise); there is no CPU fallback.
+ *   - The functions are thread-safe and may be called on different streams.
+ */
+#ifndef W4A4_H_
+#define W4A4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* w4a4_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  W4A4_OK = 0,
+  W4A4_ERR_INVALID_ARG = 1,        /* null pointer where one is required, bad enum value */
+  W4A4_ERR_UNSUPPORTED_SHAPE = 2,  /* a shape rule above is violated */
+  W4A4_ERR_MISALIGNED = 3,         /* a tensor base address is not 16-byte aligned */
+  W4A4_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+  W4A4_ERR_DEVICE_TIMEOUT = 5,     /* a kernel gave up a bounded wait (see w4a4_get_device_error) */
+  W4A4_ERR_UNSUPPORTED_DEVICE = 6, /* current device is not sm_100 */
+  W4A4_ERR_WORKSPACE = 7           /* workspace missing or smaller than *_workspace_bytes() */
+} w4a4_status;
+
+/* Version as major * 10000 + minor * 100 + patch. */
+int w4a4_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* w4a4_status_string(w4a4_status status);
+
+/* ---------------------------------------------------------------- W4A4 */
+
+/* Offline weight preparation (rotate + per-output-channel INT4 quantize +
+ * pack).  Source: "Load Diffusion Model INT4 (W4A4)" (comfy.icu), intro and
+ * "on_the_fly_quantization" (quantize BF16/FP16 weights on load).
+ *   W        bf16 [N, K] (nn.Linear layout; FP8 checkpoints must be
+ *            dequantized by the caller first)
+ *   Wq       out: uint8 [N, K/2] packed codes
+ *   w_scale  out: fp32 [N]
+ */
+w4a4_status w4a4_quantize_weights(const void* W, int N, int K, int group, uint8_t* Wq, float* w_scale,
+                                  w4a4_stream_t stream);
+
+/* On-the-fly activation path: rotate + per-token INT4 quantize + pack, and
+ * the low-rank down-projection T = X L1 when rank > 0.  Source: "W4A4 and
+ * W4A8: The New Quantization Toolkit" (renderbob.io), "Decoding the notation";
+ * "Krea 2 Turbo - SVDQuant" (sweettea.co), "What's included".
+ *   X        bf16 [M, K]
+ *   Xq       out: uint8 [M, K/2] packed codes
+ *   x_scale  out: fp32 [M]
+ *   L1       bf16 [K, rank] or NULL when rank == 0
+ *   T        out: bf16 [M, rank] or NULL when rank == 0
+ */
+w4a4_status w4a4_rotate_quantize_act(const void* X, int M, int K, int group, uint8_t* Xq, float* x_scale,
+                                     const void* L1, int rank, void* T, w4a4_stream_t stream);
+
+/* INT4 GEMM with the fused dequant + low-rank + bias epilogue.  Source:
+ * "Load Diffusion Model INT4 (W4A4)" (comfy.icu), intro (tensor-core matmul
+ * at 4 bit); "Krea 2 Turbo - SVDQuant" (sweettea.co), "What's included"
+ * (parallel low-rank branch).
+ *   Xq, x_scale  as produced by w4a4_rotate_quantize_act
+ *   Wq, w_scale  as produced by w4a4_quantize_weights (same group)
+ *   T            bf16 [M, rank] or NULL when rank == 0
+ *   L2           bf16 [rank, N] or NULL when rank == 0
+ *   bias         bf16 [N] or NULL
+ *   Y            out: bf16 [M, N]
+ *   acc_debug    out: int32 [M, N] exact integer accumulators, or NULL
+ */
+w4a4_status w4a4_gemm(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale, int M,
+                      int N, int K, int group, const void* T, const void* L2, int rank, const void* bias, void* Y,
+                      int32_t* acc_debug, w4a4_stream_t stream);
+
+/* Bytes of device workspace w4a4_linear needs: packed codes [M, K/2], scales
+ * [M] and T [M, rank], each 256-byte aligned.  Returns 0 for invalid sizes. */
+size_t w4a4_workspace_bytes(int M, int K, int rank);
+
+/* The whole layer: w4a4_rotate_quantize_act into `workspace`, then w4a4_gemm.
+ *   X bf16 [M, K]; Wq, w_scale from w4a4_quantize_weights; L1 [K, rank],
+ *   L2 [rank, N] (NULL when rank == 0); bias [N] or NULL; Y out bf16 [M, N];
+ *   workspace: device memory of at least w4a4_workspace_bytes(M, K, rank)
+ *   bytes, 256-byte aligned, owned by the caller; it must not be used by
+ *   another call that may run concurrently on the GPU.
+ */
+w4a4_status w4a4_linear(const void* X, const uint8_t* Wq, const float* w_scale, int M, int N, int K, int group,
+                        const void* L1, const void* L2, int rank, const void* bias, void* Y, void* workspace,
+                        size_t workspace_bytes, w4a4_stream_t stream);
+
+/* ---------------------------------------------------------------- W8A8 */
+/* The INT8 path for sensitive layers ("ComfyUI-INT4-Fast" (kongchang.com),
+ * "Per-Layer Dynamic Routing"; "W4A4 and W4A8" (renderbob.io), "How the
+ * toolkit tells you to choose": int8 is the W8A8 path).  Same rotation and
+ * scaling with qmax = 127, codes stored unpacked as int8 [rows, K], no
+ * low-rank branch. */
+w4a4_status w8a8_quantize_weights(const void* W, int N, int K, int group, int8_t* Wq, float* w_scale,
+                                  w4a4_stream_t stream);
+w4a4_status w8a8_rotate_quantize_act(const void* X, int M, int K, int group, int8_t* Xq, float* x_scale,
+                                     w4a4_stream_t stream);
+w4a4_status w8a8_gemm(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale, int M,
+                      int N, int K, int group, const void* bias, void* Y, int32_t* acc_debug,
+                      w4a4_stream_t stream);
+size_t w8a8_workspace_bytes(int M, int K);
+w4a4_status w8a8_linear(const void* X, const int8_t* Wq, const float* w_scale, int M, int N, int K, int group,
+                        const void* bias, void* Y, void* workspace, size_t workspace_bytes,
+                        w4a4_stream_t stream);
+
+/* ---------------------------------------------------------------- failures */
+/* Kernels never trap: a wait on another part of the kernel that runs past its
+ * time limit (2 s) records a code in a per-device error word and lets the
+ * kernel finish.  This call synchronises `stream`, reads the word of the
+ * current device into *code (may be NULL), clears it, and returns
+ * W4A4_ERR_DEVICE_TIMEOUT when it was non-zero, W4A4_OK otherwise. */
+w4a4_status w4a4_get_device_error(w4a4_stream_t stream, unsigned int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A4_H_ */

@@ -1,0 +1,146 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/w4a4.h declares, and rejects bad arguments with the
+documented status before launching anything."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a4_int4_quantized_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a4.h")
+
+OK, INVALID, SHAPE, MISALIGNED, CUDA, TIMEOUT, DEVICE, WORKSPACE = range(8)
+
+# fake device addresses: validation fails before any of them is dereferenced
+A = ctypes.c_void_p(0x10000)
+B = ctypes.c_void_p(0x20000)
+C = ctypes.c_void_p(0x30000)
+D = ctypes.c_void_p(0x40000)
+E = ctypes.c_void_p(0x50000)
+ODD = ctypes.c_void_p(0x10008)
+NUL = None
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_int4_quantized_b200 import build
+    build.build()
+    return w4.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b((?:w4a4|w8a8)_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = _declared_functions()
+    for n in ["w4a4_quantize_weights", "w4a4_rotate_quantize_act", "w4a4_gemm", "w4a4_linear",
+              "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
+              "w4a4_workspace_bytes", "w8a8_workspace_bytes", "w4a4_status_string", "w4a4_version",
+              "w4a4_get_device_error"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.w4a4_version() >= 100
+    for code, name in w4.STATUS.items():
+        assert lib.w4a4_status_string(code).decode() == name
+    assert lib.w4a4_status_string(99).decode() == "W4A4_ERR_UNKNOWN"
+
+
+def test_quantize_weights_validation(lib):
+    f = lib.w4a4_quantize_weights
+    assert f(NUL, 64, 256, 64, B, C, NUL) == INVALID
+    assert f(A, 64, 256, 64, NUL, C, NUL) == INVALID
+    assert f(A, 0, 256, 64, B, C, NUL) == SHAPE           # no rows
+    assert f(A, 64, 192, 64, B, C, NUL) == SHAPE          # K not a multiple of 128
+    assert f(A, 64, 256, 32, B, C, NUL) == SHAPE          # unsupported group
+    assert f(A, 64, 256, 96, B, C, NUL) == SHAPE
+    assert f(A, 64, 65536, 128, B, C, NUL) == SHAPE       # K / 128 > 256
+    assert f(A, 64, 32768, 64, B, C, NUL) == SHAPE        # K / 64 > 256
+    assert f(ODD, 64, 256, 64, B, C, NUL) == MISALIGNED
+    assert f(A, 64, 256, 64, ODD, C, NUL) == MISALIGNED
+    assert lib.w8a8_quantize_weights(A, 64, 256, 48, B, C, NUL) == SHAPE
+
+
+def test_rotate_quantize_act_validation(lib):
+    f = lib.w4a4_rotate_quantize_act
+    assert f(A, 8, 256, 64, B, NUL, NUL, 0, NUL, NUL) == INVALID
+    assert f(A, 8, 256, 64, B, C, NUL, 16, NUL, NUL) == INVALID        # rank without L1/T
+    assert f(A, 8, 256, 64, B, C, D, 16, NUL, NUL) == INVALID
+    assert f(A, 8, 256, 64, B, C, D, 24, E, NUL) == SHAPE              # rank not a multiple of 16
+    assert f(A, 8, 256, 64, B, C, D, 272, E, NUL) == SHAPE             # rank > 256
+    assert f(A, 8, 256, 64, B, C, ODD, 16, E, NUL) == MISALIGNED
+    assert f(A, 0, 256, 64, B, C, NUL, 0, NUL, NUL) == SHAPE
+    assert lib.w8a8_rotate_quantize_act(A, 8, 100, 0, B, C, NUL) == SHAPE
+
+
+def test_gemm_validation(lib):
+    f = lib.w4a4_gemm
+    args = [A, B, C, D, 64, 256, 256, 64, NUL, NUL, 0, NUL, E, NUL, NUL]
+    bad = list(args); bad[4] = 0
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[5] = 12                      # N not a multiple of 8
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[6] = 320
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[12] = NUL                    # no output
+    assert f(*bad) == INVALID
+    bad = list(args); bad[10] = 16                     # rank without T / L2
+    assert f(*bad) == INVALID
+    bad = list(args); bad[11] = ODD                    # misaligned bias
+    assert f(*bad) == MISALIGNED
+    bad = list(args); bad[13] = ODD                    # misaligned debug output
+    assert f(*bad) == MISALIGNED
+    assert lib.w8a8_gemm(A, B, C, D, 64, 4, 256, 128, NUL, E, NUL, NUL) == SHAPE
+
+
+def test_linear_workspace_rules(lib):
+    need = lib.w4a4_workspace_bytes(4608, 3072, 0)
+    assert need == 4608 * 1536 + 4608 * 4 + 0
+    assert lib.w4a4_workspace_bytes(3, 256, 16) == 512 + 256 + 256   # 384 B codes, 12 B scales, 96 B T
+    assert lib.w4a4_workspace_bytes(0, 256, 0) == 0
+    assert lib.w8a8_workspace_bytes(5, 256) == 1280 + 256
+    f = lib.w4a4_linear
+    args = [A, B, C, 4608, 3072, 3072, 128, NUL, NUL, 0, NUL, D, E, need, NUL]
+    bad = list(args); bad[13] = need - 1
+    assert f(*bad) == WORKSPACE
+    bad = list(args); bad[12] = NUL
+    assert f(*bad) == WORKSPACE
+    bad = list(args); bad[12] = ctypes.c_void_p(0x50010)   # not 256-byte aligned
+    assert f(*bad) == WORKSPACE
+    bad = list(args); bad[9] = 64                          # rank without L1/L2
+    assert f(*bad) == INVALID
+    g = lib.w8a8_linear
+    need8 = lib.w8a8_workspace_bytes(16, 256)
+    assert g(A, B, C, 16, 256, 256, 128, NUL, D, E, need8 - 1, NUL) == WORKSPACE
+
+
+def _cuda_visible():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.mark.skipif(_cuda_visible(), reason="only meaningful on a host without a GPU")
+def test_valid_call_without_gpu_fails_loudly(lib):
+    # all arguments valid: the call reaches the device check and must report
+    # that no CUDA device can run it (there is no CPU fallback)
+    assert lib.w4a4_quantize_weights(A, 64, 256, 64, B, C, NUL) in (CUDA, DEVICE)
+    with pytest.raises(w4.W4A4Error):
+        w4._check("w4a4_quantize_weights", lib.w4a4_quantize_weights(A, 64, 256, 64, B, C, NUL))
