@@ -18,17 +18,26 @@
 // and every product carries a factor 256, removed exactly by an arithmetic
 // shift of the int32 accumulator (|acc| <= 64 K << 2^23 for K <= 32768).
 //
-// CTA tile 128 x 256, k-block 128 codes, one CTA per SM:
-//   warps 0-3   A producers: load packed rows (256-bit loads, two k-blocks of
-//               register prefetch), widen, tcgen05.st into a TMEM ring
-//               (A is read by the MMA from tensor memory, not shared memory);
-//   warps 4-11  B producers: same for the 256 weight rows, written into a
-//               shared-memory ring in the 128-byte-swizzled K-major layout;
-//   warp 12     one elected thread issues tcgen05.mma and commits stages;
-//   warps 0-7   epilogue: tcgen05.ld of the int32 accumulator, dequant,
-//               low-rank add, bias, bf16 store (and the optional int32 copy).
+// Work decomposition: a cluster of two CTAs (one per SM of a TPC) owns a
+// 256 x 256 output tile and issues the pair form of the MMA (cta_group::2):
+// each CTA holds 128 rows of A, 128 rows (N) of B and its 128 x 256 int32
+// accumulator.  Per CTA (k-block = 128 codes):
+//   warp 8      TMA: packed A and B tiles (64-byte rows, 64-byte swizzle)
+//               into a 6-deep shared-memory ring (no multicast);
+//   warps 0-3   widen A rows (one row per thread, conflict-free 16-byte
+//               reads) and tcgen05.st them into a 4-deep TMEM ring -- A is
+//               read by the MMA from tensor memory;
+//   warps 4-7   widen B rows into a 4-deep ring in the 128-byte-swizzled
+//               K-major layout the MMA reads from shared memory;
+//   warp 9      (even CTA) one thread issues the pair MMAs and commits each
+//               stage to the barriers of both CTAs.
+//   warps 0-7   epilogue: tcgen05.ld, dequant, low-rank, bias, bf16 stores.
+// The INT8 path skips the widening: TMA writes both operands straight into
+// the 128-byte-swizzled layout and the MMA reads both from shared memory.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
-// the device error word and exits without trapping.
+// the device error word and runs to completion without trapping.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -38,36 +47,77 @@ namespace w4a4 {
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;                 // 8-bit elements per k-block
-constexpr int kStages = 6;
-constexpr int kNumAWarps = 4;
-constexpr int kNumBWarps = 8;
-constexpr int kMmaWarp = kNumAWarps + kNumBWarps;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
-constexpr int kBStageBytes = BN * BK;   // 32 KB of widened codes
-constexpr uint32_t kAccCol = 0;         // int32 accumulator: columns [0, 256)
-constexpr uint32_t kACol0 = 256;        // A ring: 32 columns (128 codes) per stage
-constexpr uint32_t kTmemCols = 512;
-constexpr int kSmemBytes = kStages * kBStageBytes + 1024 /*alignment slack*/ + 256 /*barriers*/;
+constexpr int BM = 128;          // A rows per CTA; the pair covers 256
+constexpr int BN = 256;          // N per pair tile
+constexpr int BNH = BN / 2;      // B rows staged per CTA
+constexpr int BK = 128;          // codes per k-block
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
 
-static_assert(kACol0 + kStages * (BK / 4) <= kTmemCols, "TMEM budget");
+// packed (INT4) path
+constexpr int PS = 6;                                // packed TMA stages
+constexpr int US = 4;                                // widened stages
+constexpr int kPkA = BM * BK / 2;                    // 8 KB
+constexpr int kPkB = BNH * BK / 2;                   // 8 KB
+constexpr int kPkStage = kPkA + kPkB;
+constexpr int kWideB = BNH * BK;                     // 16 KB
+constexpr int kPkRingBytes = PS * kPkStage;          // 96 KB
+constexpr int kWideRingBytes = US * kWideB;          // 64 KB
+// int8 path
+constexpr int S8 = 5;
+constexpr int kI8A = BM * BK;                        // 16 KB
+constexpr int kI8B = BNH * BK;                       // 16 KB
+constexpr int kI8Stage = kI8A + kI8B;
+
+constexpr uint32_t kAccCol = 0;                      // int32 accumulator: columns [0, 256)
+constexpr uint32_t kACol0 = 256;                     // A ring: 32 columns per stage
+constexpr uint32_t kTmemCols = 512;
+
+// epilogue: per-warp double-buffered 32 x 32 bf16 staging tiles for TMA
+// stores (64-byte rows, 64-byte swizzle), then the tile's weight scales and
+// bias in fp32
+constexpr int kStageTile = 32 * 32 * 2;               // 2 KB
+constexpr int kOutStageBytes = 8 * 2 * kStageTile;     // 32 KB
+constexpr int kVecBytes = 2 * BN * 4;                  // 2 KB
+constexpr int kBarBytes = 512;
+template <bool PACKED>
+constexpr int ring_bytes() { return PACKED ? kPkRingBytes + kWideRingBytes : S8 * kI8Stage; }
+template <bool PACKED>
+constexpr int data_bytes() { return ring_bytes<PACKED>() + kOutStageBytes + kVecBytes; }
+template <bool PACKED>
+constexpr int smem_bytes() { return data_bytes<PACKED>() + kBarBytes + 1024; }
+static_assert(smem_bytes<true>() <= 232448 && smem_bytes<false>() <= 232448, "shared memory budget");
+
+static_assert(kACol0 + US * (BK / 4) <= kTmemCols, "TMEM budget");
 
 struct Params {
   GemmArgs a;
   unsigned int* err;
 };
 
-__device__ __forceinline__ void ld_nc_256(const void* p, uint4& lo, uint4& hi) {
-  asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
-               : "l"(p));
-}
+struct Barriers {
+  uint64_t tma_full[8];
+  uint64_t tma_empty[8];
+  uint64_t wfull[8];     // this CTA's widened stage is complete (8 warp arrivals)
+  uint64_t full[8];      // even CTA: the odd CTA's stage is complete (1 relay arrival)
+  uint64_t empty[8];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+};
+static_assert(sizeof(Barriers) <= kBarBytes, "barrier block");
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 // 16 packed bytes (32 codes) -> 32 widened bytes (two 16-byte chunks).
@@ -85,71 +135,150 @@ __device__ __forceinline__ void widen16(const uint4 p, uint4& c0, uint4& c1) {
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
 template <bool PACKED>
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const Params prm) {
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY) {
   const GemmArgs& p = prm.a;
-  constexpr int V = PACKED ? 4 : 8;               // 16-byte vectors per row per k-block
-  constexpr int kShift = PACKED ? 8 : 0;          // widened products carry 2^8
+  constexpr int kShift = PACKED ? 8 : 0;  // widened products carry 2^8
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (sbase - raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kBStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  Barriers* bar = reinterpret_cast<Barriers*>(smem_raw + (sbase - raw) + data_bytes<PACKED>());
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * BM;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int m_cta = (pair / n_tiles) * (2 * BM) + (int)rank * BM;   // this CTA's A rows
+  const int n_pair = (pair % n_tiles) * BN;                          // pair's N columns
+  const int n_cta = n_pair + (int)rank * BNH;                        // this CTA's B rows
   const int nk = p.K / BK;
-  const long row_bytes = PACKED ? p.K / 2 : p.K;
 
-  if (warp == kMmaWarp) {
+  if (warp == kTmaWarp) {
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
-        mbar_init(&full[s], (kNumAWarps + kNumBWarps) * 32);
-        mbar_init(&empty[s], 1);
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      prefetch_tmap(&tmY);
+      for (int s = 0; s < 8; ++s) {
+        mbar_init(&bar->tma_full[s], 1);
+        mbar_init(&bar->tma_empty[s], PACKED ? 8 : 1);
+        mbar_init(&bar->wfull[s], 8);
+        mbar_init(&bar->full[s], 1);
+        mbar_init(&bar->empty[s], 1);
       }
-      mbar_init(acc_full, 1);
+      mbar_init(&bar->acc_full, 1);
       fence_mbar_init();
     }
     __syncwarp();
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&bar->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem = bar->tmem_base;
 
-  if (warp < kMmaWarp) {
-    // ------------------------------------------------------------ producers
-    const bool is_a = warp < kNumAWarps;
-    const int r = is_a ? warp * 32 + lane : (warp - kNumAWarps) * 32 + lane;
-    const long g_row = is_a ? (long)m0 + r : (long)n0 + r;
-    const bool ok = g_row < (is_a ? p.M : p.N);
-    const uint8_t* src = (is_a ? p.A : p.B) + (ok ? g_row : 0) * row_bytes;
-    const uint32_t a_taddr = tmem + ((uint32_t)(warp * 32) << 16) + kACol0;
-    const uint32_t b_row = sbase + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
-    const uint32_t sw = (uint32_t)(r & 7);
-
-    auto load = [&](uint4 (&buf)[V], int kb) {
-      if (ok && kb < nk) {
-        const uint8_t* q = src + (long)kb * (V * 16);
-#pragma unroll
-        for (int v = 0; v < V; v += 2) ld_nc_256(q + v * 16, buf[v], buf[v + 1]);
-      } else {
-#pragma unroll
-        for (int v = 0; v < V; ++v) buf[v] = make_uint4(0u, 0u, 0u, 0u);
+  if (warp == kTmaWarp) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      constexpr int NS = PACKED ? PS : S8;
+      constexpr int kStageBytes = PACKED ? kPkStage : kI8Stage;
+      constexpr int kABytes = PACKED ? kPkA : kI8A;
+      constexpr int kColBytes = PACKED ? BK / 2 : BK;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % NS;
+        if (!mbar_wait(&bar->tma_empty[s], ((uint32_t)(kb / NS) & 1u) ^ 1u)) {
+          set_device_error(prm.err, kDevErrTimeoutEmpty);
+          break;
+        }
+        const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
+        mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
+        tma_load_2d(dst, &tmA, kb * kColBytes, m_cta, &bar->tma_full[s]);
+        tma_load_2d(dst + kABytes, &tmB, kb * kColBytes, n_cta, &bar->tma_full[s]);
       }
-    };
-    auto produce = [&](int kb, const uint4 (&cur)[V]) -> bool {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!mbar_wait(&empty[s], ph ^ 1u)) {
+    }
+  } else if (warp == kMmaWarp) {
+    if (!leader && lane == 0) {
+      // relay: one cluster-scope arrival per stage tells the even CTA that
+      // this CTA's operands are in place (TMA landed, or all 8 widen warps
+      // done), instead of one per warp
+      constexpr int NS = PACKED ? US : S8;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % NS;
+        if (!mbar_wait(PACKED ? &bar->wfull[s] : &bar->tma_full[s], (uint32_t)(kb / NS) & 1u)) {
+          set_device_error(prm.err, kDevErrTimeoutFull);
+          break;
+        }
+        mbar_arrive_cluster(&bar->full[s], 0);
+      }
+    }
+    if (leader && lane == 0) {
+      // ---------------------------------------------------------------- MMA
+      constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
+      bool ok = true;
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        if (PACKED) {
+          const int u = kb % US;
+          const uint32_t ph = (uint32_t)(kb / US) & 1u;
+          if (!mbar_wait(&bar->wfull[u], ph) || !mbar_wait_cluster(&bar->full[u], ph)) {
+            set_device_error(prm.err, kDevErrTimeoutFull);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_stage = sbase + (uint32_t)(kPkRingBytes + u * kWideB);
+#pragma unroll
+          for (int ks = 0; ks < BK / 32; ++ks)
+            mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(u * (BK / 4) + ks * 8),
+                           smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc, (kb | ks) != 0 ? 1u : 0u);
+          tc_commit_pair_mc(&bar->empty[u], 0x3);
+        } else {
+          const int s = kb % S8;
+          const uint32_t ph = (uint32_t)(kb / S8) & 1u;
+          if (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait_cluster(&bar->full[s], ph)) {
+            set_device_error(prm.err, kDevErrTimeoutFull);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_stage = sbase + (uint32_t)(s * kI8Stage);
+#pragma unroll
+          for (int ks = 0; ks < BK / 32; ++ks)
+            mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
+                           smem_desc_kmajor_sw128(a_stage + kI8A + (uint32_t)(ks * 32)), idesc,
+                           (kb | ks) != 0 ? 1u : 0u);
+          tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
+        }
+      }
+      tc_commit_pair_mc(&bar->acc_full, 0x3);
+      if (!mbar_wait(&bar->acc_full, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
+    }
+  } else if (PACKED) {
+    // ---------------------------------------------------------------- widen
+    const bool is_a = warp < 4;
+    const int r = (warp & 3) * 32 + lane;                  // row within this CTA's tile
+    const uint32_t sw64 = (uint32_t)((r >> 1) & 3);
+    const uint32_t sw128 = (uint32_t)(r & 7);
+    const uint32_t a_taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + kACol0;
+    const uint32_t wide_row = sbase + (uint32_t)(kPkRingBytes + (r >> 3) * 1024 + (r & 7) * 128);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int ps = kb % PS;
+      const int u = kb % US;
+      if (!mbar_wait(&bar->tma_full[ps], (uint32_t)(kb / PS) & 1u)) {
+        set_device_error(prm.err, kDevErrTimeoutFull);
+        break;
+      }
+      const uint32_t src = sbase + (uint32_t)(ps * kPkStage + (is_a ? 0 : kPkA) + r * (BK / 2));
+      uint4 pk[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ sw64) << 4));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->tma_empty[ps]);
+      if (!mbar_wait(&bar->empty[u], ((uint32_t)(kb / US) & 1u) ^ 1u)) {
         set_device_error(prm.err, kDevErrTimeoutEmpty);
-        return false;
+        break;
       }
       tc_fence_after();
       if (is_a) {
@@ -157,102 +286,68 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const Params prm) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 c0, c1;
-          if (PACKED) {
-            widen16(cur[c], c0, c1);
-          } else {
-            c0 = cur[2 * c];
-            c1 = cur[2 * c + 1];
-          }
+          widen16(pk[c], c0, c1);
           regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
           regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
         }
-        tmem_st_32x32b_x32(a_taddr + (uint32_t)(s * (BK / 4)), regs);
+        tmem_st_32x32b_x32(a_taddr + (uint32_t)(u * (BK / 4)), regs);
         tmem_wait_st();
         tc_fence_before();
       } else {
-        const uint32_t row = b_row + (uint32_t)(s * kBStageBytes);
+        const uint32_t row = wide_row + (uint32_t)(u * kWideB);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 c0, c1;
-          if (PACKED) {
-            widen16(cur[c], c0, c1);
-          } else {
-            c0 = cur[2 * c];
-            c1 = cur[2 * c + 1];
-          }
-          st_shared_v4(row + (((uint32_t)(2 * c) ^ sw) << 4), c0);
-          st_shared_v4(row + (((uint32_t)(2 * c + 1) ^ sw) << 4), c1);
+          widen16(pk[c], c0, c1);
+          st_shared_v4(row + ((((uint32_t)(2 * c)) ^ sw128) << 4), c0);
+          st_shared_v4(row + ((((uint32_t)(2 * c + 1)) ^ sw128) << 4), c1);
         }
         fence_proxy_async_smem();
       }
-      mbar_arrive(&full[s]);
-      return true;
-    };
-
-    uint4 b0[V], b1[V], b2[V];
-    load(b0, 0);
-    load(b1, 1);
-    for (int kb = 0; kb < nk; kb += 3) {
-      load(b2, kb + 2);
-      if (!produce(kb, b0)) break;
-      if (kb + 1 >= nk) break;
-      load(b0, kb + 3);
-      if (!produce(kb + 1, b1)) break;
-      if (kb + 2 >= nk) break;
-      load(b1, kb + 4);
-      if (!produce(kb + 2, b2)) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->wfull[u]);
     }
-  } else if (lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc = idesc_i8(BM, BN);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!mbar_wait(&full[s], ph)) {
-        set_device_error(prm.err, kDevErrTimeoutFull);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t b_stage = sbase + (uint32_t)(s * kBStageBytes);
-#pragma unroll
-      for (int ks = 0; ks < BK / 32; ++ks) {
-        const uint64_t bdesc = smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32));
-        mma_i8_ts(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8), bdesc, idesc,
-                  (kb | ks) != 0 ? 1u : 0u);
-      }
-      tc_commit(&empty[s]);
-    }
-    tc_commit(acc_full);
-    if (!mbar_wait(acc_full, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
   }
 
   // ------------------------------------------------------------ epilogue
   if (warp < 8) {
     const int quad = warp & 3;
     const int half = warp >> 2;
-    if (!mbar_wait(acc_full, 0)) set_device_error(prm.err, kDevErrTimeoutAcc);
+    const uint32_t stage_out = sbase + (uint32_t)(ring_bytes<PACKED>() + warp * 2 * kStageTile);
+    float* s_sw = reinterpret_cast<float*>(smem_raw + (sbase - raw) + ring_bytes<PACKED>() + kOutStageBytes);
+    float* s_bias = s_sw + BN;
+    {
+      // this tile's weight scales and bias, staged once for all 256 threads
+      const int j = threadIdx.x;  // 0..255
+      const int n = n_pair + j;
+      s_sw[j] = n < p.N ? __ldg(p.b_scale + n) : 0.0f;
+      s_bias[j] = (p.bias && n < p.N) ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f;
+    }
+    named_barrier_sync(1, 256);
+    if (!mbar_wait(&bar->acc_full, 0)) set_device_error(prm.err, kDevErrTimeoutAcc);
     tc_fence_after();
-    const long m = (long)m0 + quad * 32 + lane;
+    const int m_row0 = m_cta + quad * 32;
+    const long m = (long)m_row0 + lane;
     const bool mok = m < p.M;
     const float sa = mok ? __ldg(p.a_scale + m) : 0.0f;
+    const uint32_t sw64 = (uint32_t)((lane >> 1) & 3);
 #pragma unroll 1
     for (int ch = 0; ch < 4; ++ch) {
       const int c0 = half * 128 + ch * 32;
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kAccCol + (uint32_t)c0, v);
       tmem_wait_ld();
-      const int n = n0 + c0;
+      const int n = n_pair + c0;
+      if (n >= p.N) continue;  // warp-uniform
       const int nv = min(32, p.N - n);
-      if (nv <= 0 || !mok) continue;
       float y[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int acc = static_cast<int>(v[j]) >> kShift;
         v[j] = static_cast<uint32_t>(acc);
-        const float sw = j < nv ? __ldg(p.b_scale + n + j) : 0.0f;
-        y[j] = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa), sw), p.inv_group);
+        y[j] = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa), s_sw[c0 + j]), p.inv_group);
       }
-      if (p.rank > 0) {
+      if (p.rank > 0 && mok) {
         const uint16_t* trow = p.T + m * p.rank;
 #pragma unroll 1
         for (int jj = 0; jj < p.rank; ++jj) {
@@ -265,8 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const Params prm) {
       }
       if (p.bias) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nv) y[j] = __fadd_rn(y[j], bf16_bits_to_float(__ldg(p.bias + n + j)));
+        for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], s_bias[c0 + j]);
       }
       uint32_t o[16];
 #pragma unroll
@@ -274,26 +368,79 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const Params prm) {
         __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
         o[j] = *reinterpret_cast<uint32_t*>(&h);
       }
-      uint4* dst = reinterpret_cast<uint4*>(p.Y + m * p.N + n);
+      // stage the warp's 32 x 32 tile and let TMA write it (rows past M and
+      // columns past N are dropped by the tensor map bounds)
+      const uint32_t buf = stage_out + (uint32_t)((ch & 1) * kStageTile);
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (8 * c < nv) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-      if (p.acc_debug) {
+        st_shared_v4(buf + (uint32_t)(lane * 64) + ((((uint32_t)c) ^ sw64) << 4),
+                     make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tmY, buf, n, m_row0);
+        bulk_commit();
+      }
+      if (p.acc_debug && mok) {
         uint4* dd = reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n);
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           if (4 * c < nv) dd[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
       }
     }
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    __syncwarp();
+  cluster_sync();
+  if (warp == kTmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// Row-major uint8 matrix [rows, cols] as a 2-D tensor map with a
+// (box_cols x box_rows) box; rows past the end read as zero.
+bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                  uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major bf16 matrix [rows, cols] as a 2-D tensor map (box_cols x box_rows).
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <bool PACKED>
@@ -303,13 +450,35 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !configured[dev]) {
-    e = cudaFuncSetAttribute(gemm_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(gemm_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<PACKED>());
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
+  CUtensorMap tA, tB;
+  const uint64_t row_bytes = PACKED ? (uint64_t)a.K / 2 : (uint64_t)a.K;
+  const uint32_t box_cols = PACKED ? BK / 2 : BK;
+  const CUtensorMapSwizzle swz = PACKED ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap tY;
+  if (!make_tmap_u8(&tA, a.A, (uint64_t)a.M, row_bytes, box_cols, BM, swz) ||
+      !make_tmap_u8(&tB, a.B, (uint64_t)a.N, row_bytes, box_cols, BNH, swz) ||
+      !make_tmap_bf16(&tY, a.Y, (uint64_t)a.M, (uint64_t)a.N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  const int pairs = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<PACKED>();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   Params prm{a, err};
-  gemm_kernel<PACKED><<<grid, kThreads, kSmemBytes, st>>>(prm);
+  e = cudaLaunchKernelEx(&cfg, gemm_kernel<PACKED>, prm, tA, tB, tY);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
