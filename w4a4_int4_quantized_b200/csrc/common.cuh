@@ -100,12 +100,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// Arrive (release, cluster scope) on the barrier at the same shared-memory
-// offset in CTA `rank` of this cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
+// Arrive on the barrier at the same shared-memory offset in CTA `rank` of
+// this cluster (default release semantics, as the 2-CTA tensor-core
+// pipelines use for producer -> MMA hand-off inside a CTA pair).
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -56,14 +56,14 @@ constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 
 // packed (INT4) path
-constexpr int PS = 6;                                // packed TMA stages
-constexpr int US = 4;                                // widened stages
+constexpr int PS = 5;                                // packed TMA stages
+constexpr int US = 6;                                // widened stages
 constexpr int kPkA = BM * BK / 2;                    // 8 KB
 constexpr int kPkB = BNH * BK / 2;                   // 8 KB
 constexpr int kPkStage = kPkA + kPkB;
 constexpr int kWideB = BNH * BK;                     // 16 KB
-constexpr int kPkRingBytes = PS * kPkStage;          // 96 KB
-constexpr int kWideRingBytes = US * kWideB;          // 64 KB
+constexpr int kPkRingBytes = PS * kPkStage;          // 80 KB
+constexpr int kWideRingBytes = US * kWideB;          // 96 KB
 // int8 path
 constexpr int S8 = 5;
 constexpr int kI8A = BM * BK;                        // 16 KB
@@ -99,8 +99,7 @@ struct Params {
 struct Barriers {
   uint64_t tma_full[8];
   uint64_t tma_empty[8];
-  uint64_t wfull[8];     // this CTA's widened stage is complete (8 warp arrivals)
-  uint64_t full[8];      // even CTA: the odd CTA's stage is complete (1 relay arrival)
+  uint64_t full[8];      // even CTA: a stage is complete in both CTAs
   uint64_t empty[8];
   uint64_t acc_full;
   uint32_t tmem_base;
@@ -164,8 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < 8; ++s) {
         mbar_init(&bar->tma_full[s], 1);
         mbar_init(&bar->tma_empty[s], PACKED ? 8 : 1);
-        mbar_init(&bar->wfull[s], 8);
-        mbar_init(&bar->full[s], 1);
+        mbar_init(&bar->full[s], PACKED ? 16 : 1);  // 8 widen warps per CTA, or 1 relay
         mbar_init(&bar->empty[s], 1);
       }
       mbar_init(&bar->acc_full, 1);
@@ -200,18 +198,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    if (!leader && lane == 0) {
-      // relay: one cluster-scope arrival per stage tells the even CTA that
-      // this CTA's operands are in place (TMA landed, or all 8 widen warps
-      // done), instead of one per warp
-      constexpr int NS = PACKED ? US : S8;
+    if (!PACKED && !leader && lane == 0) {
+      // relay: tell the even CTA when this CTA's operand tiles have landed
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % NS;
-        if (!mbar_wait(PACKED ? &bar->wfull[s] : &bar->tma_full[s], (uint32_t)(kb / NS) & 1u)) {
+        const int s = kb % S8;
+        if (!mbar_wait(&bar->tma_full[s], (uint32_t)(kb / S8) & 1u)) {
           set_device_error(prm.err, kDevErrTimeoutFull);
           break;
         }
-        mbar_arrive_cluster(&bar->full[s], 0);
+        mbar_arrive_remote(&bar->full[s], 0);
       }
     }
     if (leader && lane == 0) {
@@ -221,8 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < nk && ok; ++kb) {
         if (PACKED) {
           const int u = kb % US;
-          const uint32_t ph = (uint32_t)(kb / US) & 1u;
-          if (!mbar_wait(&bar->wfull[u], ph) || !mbar_wait_cluster(&bar->full[u], ph)) {
+          if (!mbar_wait(&bar->full[u], (uint32_t)(kb / US) & 1u)) {
             set_device_error(prm.err, kDevErrTimeoutFull);
             ok = false;
             break;
@@ -237,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int s = kb % S8;
           const uint32_t ph = (uint32_t)(kb / S8) & 1u;
-          if (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait_cluster(&bar->full[s], ph)) {
+          if (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait(&bar->full[s], ph)) {
             set_device_error(prm.err, kDevErrTimeoutFull);
             ok = false;
             break;
@@ -305,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->wfull[u]);
+      if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
     }
   }
 

@@ -57,7 +57,7 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-constexpr int kStages = 3;
+constexpr int kStages = 2;  // 3 CTAs per SM each keep one block in flight
 
 // Shared-memory stride of one staged group: g bf16 plus 16 bytes of padding,
 // so that the 16-byte reads of eight consecutive threads (eight consecutive
@@ -65,26 +65,65 @@ constexpr int kStages = 3;
 template <int G>
 constexpr int group_stride() { return G * 2 + 16; }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Codes of 16 elements (8 float2 pairs) -> bw: INT4 {.x word, .y word}
+// (value j of a word in bits 4j..4j+3), INT8 {.x lo, .x hi, .y lo, .y hi}.
+// The fast form brackets each quotient between two fused multiply-adds and
+// ORs any disagreement into `bad`; the exact form uses IEEE division.
+template <bool INT4, bool EXACT>
+__device__ __forceinline__ void quantize_block8(const float2* P8, float2 ih, float2 il, float s, uint32_t* bw,
+                                                uint32_t& bad) {
+  const float2 mg = make_float2(kMagic, kMagic);
+  uint32_t tx[8], ty[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (EXACT) {
+      tx[j] = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(P8[j].x, s)), kMagic));
+      ty[j] = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(P8[j].y, s)), kMagic));
+    } else {
+      const float2 th = __ffma2_rn(P8[j], ih, mg);
+      const float2 tl = __ffma2_rn(P8[j], il, mg);
+      tx[j] = __float_as_uint(th.x);
+      ty[j] = __float_as_uint(th.y);
+      bad |= (tx[j] ^ __float_as_uint(tl.x)) | (ty[j] ^ __float_as_uint(tl.y));
+    }
+  }
+  if (INT4) {
+    bw[0] = pack_nibbles8(tx);
+    bw[1] = pack_nibbles8(ty);
+  } else {
+    bw[0] = pack_bytes4(tx[0], tx[1], tx[2], tx[3]);
+    bw[1] = pack_bytes4(tx[4], tx[5], tx[6], tx[7]);
+    bw[2] = pack_bytes4(ty[0], ty[1], ty[2], ty[3]);
+    bw[3] = pack_bytes4(ty[4], ty[5], ty[6], ty[7]);
+  }
+}
+
 // Persistent CTAs walk blocks of R consecutive rows.  Blocks are staged in a
 // 3-deep shared-memory ring with cp.async (coalesced 16-byte copies, no
 // registers held while in flight), so the loads of the next blocks overlap
-// the rotation and quantization of the current one.
-template <int G, bool ROT, int QMAX>
-__global__ void __launch_bounds__(256) rotate_quantize_kernel(const uint16_t* __restrict__ X, int M, int K,
-                                                              int rows_per_blk, uint8_t* __restrict__ out,
-                                                              float* __restrict__ scale) {
+// the rotation and quantization of the current one.  One thread owns one
+// group; its g values go from shared memory straight into float2 registers.
+template <int G, bool ROT, int QMAX, int MAXT>
+__global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
+    rotate_quantize_kernel(const uint16_t* __restrict__ X, int M, int K, int rows_per_blk, uint8_t* __restrict__ out,
+                           float* __restrict__ scale) {
   constexpr int HALF = G / 2;
   constexpr bool INT4 = (QMAX == 7);
   constexpr int GS = group_stride<G>();
   extern __shared__ __align__(16) uint8_t stage_mem[];
-  __shared__ unsigned int rowmax[2][256];
+  __shared__ unsigned int rowmax[2][MAXT];
 
   const int gpr = K / G;
   const int tid = threadIdx.x;
   const int lr = tid / gpr;
   const int grp = tid - lr * gpr;
-  const int groups_per_blk = rows_per_blk * gpr;
-  const int stage_bytes = groups_per_blk * GS;
+  const int stage_bytes = rows_per_blk * gpr * GS;
   const int nblk = (M + rows_per_blk - 1) / rows_per_blk;
   const uint32_t stage0 = smem_u32(stage_mem);
   constexpr int CPG = G / 8;  // 16-byte chunks per group
@@ -103,7 +142,7 @@ __global__ void __launch_bounds__(256) rotate_quantize_kernel(const uint16_t* __
     cp_async_commit();
   };
 
-  if (tid < 256) rowmax[0][tid] = 0u;
+  rowmax[0][tid] = 0u;
 #pragma unroll
   for (int it = 0; it < kStages - 1; ++it) issue(it);
 
@@ -121,23 +160,21 @@ __global__ void __launch_bounds__(256) rotate_quantize_kernel(const uint16_t* __
     float2 P[HALF];  // P[i] = (y_i, y_{i+HALF})
     if (active) {
       const uint32_t gsrc = stage0 + (uint32_t)((it % kStages) * stage_bytes + tid * GS);
-      uint32_t w[G / 2];
 #pragma unroll
       for (int i = 0; i < G / 8; ++i) {
         uint4 t;
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(t.x), "=r"(t.y), "=r"(t.z), "=r"(t.w)
                      : "r"(gsrc + i * 16));
-        w[4 * i + 0] = t.x;
-        w[4 * i + 1] = t.y;
-        w[4 * i + 2] = t.z;
-        w[4 * i + 3] = t.w;
-      }
+        // elements 8i .. 8i+7 of the group
+        const uint32_t wv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-      for (int i = 0; i < HALF; ++i) {
-        const uint32_t a = w[i / 2], b = w[(i + HALF) / 2];
-        P[i].x = (i & 1) ? bf16hi(a) : bf16lo(a);
-        P[i].y = (i & 1) ? bf16hi(b) : bf16lo(b);
+        for (int q = 0; q < 8; ++q) {
+          const int e = 8 * i + q;
+          const float f = (q & 1) ? bf16hi(wv[q / 2]) : bf16lo(wv[q / 2]);
+          if (e < HALF) P[e].x = f;
+          else P[e - HALF].y = f;
+        }
       }
       if (ROT) {
         // stages h = 1 .. HALF/2: pairs (i, i+h) sit in different float2s
@@ -162,7 +199,7 @@ __global__ void __launch_bounds__(256) rotate_quantize_kernel(const uint16_t* __
       }
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < HALF; ++i) amax = fmaxf(amax, fmaxf(fabsf(P[i].x), fabsf(P[i].y)));
+      for (int i = 0; i < HALF; ++i) amax = max3(amax, fabsf(P[i].x), fabsf(P[i].y));
       atomicMax(&rmax[lr], __float_as_uint(amax));
     }
     __syncthreads();
@@ -178,70 +215,51 @@ __global__ void __launch_bounds__(256) rotate_quantize_kernel(const uint16_t* __
       inv_lo = __fmul_rn(inv, 1.0f - 0x1p-20f);
     }
     const float2 ih = make_float2(inv_hi, inv_hi), il = make_float2(inv_lo, inv_lo);
-    const float2 mg = make_float2(kMagic, kMagic);
 
-    constexpr int NW = INT4 ? G / 8 : G / 4;  // output words
-    uint32_t outw[NW];
-    uint32_t bad = 0u;
-#pragma unroll
-    for (int blk8 = 0; blk8 < HALF / 8; ++blk8) {
-      uint32_t tx[8], ty[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float2 th = __ffma2_rn(P[8 * blk8 + j], ih, mg);
-        const float2 tl = __ffma2_rn(P[8 * blk8 + j], il, mg);
-        tx[j] = __float_as_uint(th.x);
-        ty[j] = __float_as_uint(th.y);
-        bad |= (tx[j] ^ __float_as_uint(tl.x)) | (ty[j] ^ __float_as_uint(tl.y));
-      }
-      if (INT4) {
-        outw[blk8] = pack_nibbles8(tx);
-        outw[HALF / 8 + blk8] = pack_nibbles8(ty);
-      } else {
-        outw[2 * blk8] = pack_bytes4(tx[0], tx[1], tx[2], tx[3]);
-        outw[2 * blk8 + 1] = pack_bytes4(tx[4], tx[5], tx[6], tx[7]);
-        outw[HALF / 4 + 2 * blk8] = pack_bytes4(ty[0], ty[1], ty[2], ty[3]);
-        outw[HALF / 4 + 2 * blk8 + 1] = pack_bytes4(ty[4], ty[5], ty[6], ty[7]);
-      }
-    }
-    if (bad) {
-      // A quotient sits within 2^-20 (relative) of a rounding boundary: redo
-      // this group with the IEEE quotient the codes are defined by.
-#pragma unroll
-      for (int blk8 = 0; blk8 < HALF / 8; ++blk8) {
-        uint32_t tx[8], ty[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          tx[j] = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(P[8 * blk8 + j].x, s)), kMagic));
-          ty[j] = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(P[8 * blk8 + j].y, s)), kMagic));
-        }
-        if (INT4) {
-          outw[blk8] = pack_nibbles8(tx);
-          outw[HALF / 8 + blk8] = pack_nibbles8(ty);
-        } else {
-          outw[2 * blk8] = pack_bytes4(tx[0], tx[1], tx[2], tx[3]);
-          outw[2 * blk8 + 1] = pack_bytes4(tx[4], tx[5], tx[6], tx[7]);
-          outw[HALF / 4 + 2 * blk8] = pack_bytes4(ty[0], ty[1], ty[2], ty[3]);
-          outw[HALF / 4 + 2 * blk8 + 1] = pack_bytes4(ty[4], ty[5], ty[6], ty[7]);
-        }
-      }
-    }
+    // Codes leave in 16-byte chunks as soon as they are complete: SB blocks of
+    // 8 pairs fill one chunk of .x-lane codes and one of .y-lane codes.  A
+    // block whose quotients come within 2^-20 (relative) of a rounding
+    // boundary is redone at once with the IEEE quotient the codes are
+    // defined by.
+    constexpr int SB = INT4 ? 4 : 2;
+    constexpr int YCH = INT4 ? HALF / 32 : HALF / 16;  // first chunk of .y codes
     const long row_bytes = INT4 ? K / 2 : K;
     uint4* dst = reinterpret_cast<uint4*>(out + row * row_bytes + (long)grp * (INT4 ? G / 2 : G));
 #pragma unroll
-    for (int i = 0; i < NW / 4; ++i)
-      dst[i] = make_uint4(outw[4 * i], outw[4 * i + 1], outw[4 * i + 2], outw[4 * i + 3]);
+    for (int c = 0; c < HALF / (8 * SB); ++c) {
+      uint32_t w[2 * SB * (INT4 ? 1 : 2)];  // .x words then .y words
+#pragma unroll
+      for (int b = 0; b < SB; ++b) {
+        const int blk8 = c * SB + b;
+        uint32_t bw[INT4 ? 2 : 4];
+        uint32_t bad = 0u;
+        quantize_block8<INT4, false>(P + 8 * blk8, ih, il, s, bw, bad);
+        if (bad) quantize_block8<INT4, true>(P + 8 * blk8, ih, il, s, bw, bad);
+        if (INT4) {
+          w[b] = bw[0];
+          w[SB + b] = bw[1];
+        } else {
+          w[2 * b] = bw[0];
+          w[2 * b + 1] = bw[1];
+          w[2 * SB + 2 * b] = bw[2];
+          w[2 * SB + 2 * b + 1] = bw[3];
+        }
+      }
+      dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[YCH + c] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
   }
   cp_async_wait<0>();
 }
 
-template <int G, bool ROT, int QMAX>
-cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scale, cudaStream_t st) {
+template <int G, bool ROT, int QMAX, int MAXT>
+cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* scale, cudaStream_t st) {
   const int gpr = K / G;
-  const int rows_per_blk = gpr >= 128 ? 1 : 128 / gpr;
+  const int rows_per_blk = gpr >= MAXT ? 1 : MAXT / gpr;
   const int threads = ((rows_per_blk * gpr + 31) / 32) * 32;
+  if (threads > MAXT) return cudaErrorInvalidConfiguration;
   const int smem = kStages * rows_per_blk * gpr * group_stride<G>();
-  auto kern = rotate_quantize_kernel<G, ROT, QMAX>;
+  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT>;
   static int attr_set[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -258,6 +276,14 @@ cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scal
   const int grid = min(nblk, sms * max(per_sm, 1));
   kern<<<grid, threads, smem, st>>>(X, M, K, rows_per_blk, out, scale);
   return cudaGetLastError();
+}
+
+// Rows of up to 128 groups run in 128-thread CTAs (three per SM); wider rows
+// (K / g > 128) in 256-thread CTAs, one group per thread either way.
+template <int G, bool ROT, int QMAX>
+cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scale, cudaStream_t st) {
+  if (K / G <= 128) return launch_rq_t<G, ROT, QMAX, 128>(X, M, K, out, scale, st);
+  return launch_rq_t<G, ROT, QMAX, 256>(X, M, K, out, scale, st);
 }
 
 }  // namespace
