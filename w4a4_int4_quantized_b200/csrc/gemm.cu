@@ -32,10 +32,15 @@
 //   warp 9      (even CTA) one thread issues the pair MMAs and commits each
 //               stage to the barriers of both CTAs.
 //   warps 0-7   epilogue: tcgen05.ld, dequant, low-rank, bias, bf16 stores.
+// The kernel is persistent: one pair per TPC walks its output tiles, and the
+// TMA and widen stages run ahead into the next tile while the epilogue of the
+// current one drains the (single) accumulator.
 // The INT8 path skips the widening: TMA writes both operands straight into
 // the 128-byte-swizzled layout and the MMA reads both from shared memory.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
 // the device error word and runs to completion without trapping.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -51,9 +56,9 @@ constexpr int BM = 128;          // A rows per CTA; the pair covers 256
 constexpr int BN = 256;          // N per pair tile
 constexpr int BNH = BN / 2;      // B rows staged per CTA
 constexpr int BK = 128;          // codes per k-block
-constexpr int kThreads = 320;    // 10 warps
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 576;    // 18 warps
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
 
 // packed (INT4) path
 constexpr int PS = 5;                                // packed TMA stages
@@ -79,7 +84,7 @@ constexpr uint32_t kTmemCols = 512;
 // bias in fp32
 constexpr int kStageTile = 32 * 32 * 2;               // 2 KB
 constexpr int kOutStageBytes = 8 * 2 * kStageTile;     // 32 KB
-constexpr int kVecBytes = 2 * BN * 4;                  // 2 KB
+constexpr int kVecBytes = 2 * 2 * BN * 4;              // 4 KB (two tiles)
 constexpr int kBarBytes = 512;
 template <bool PACKED>
 constexpr int ring_bytes() { return PACKED ? kPkRingBytes + kWideRingBytes : S8 * kI8Stage; }
@@ -102,6 +107,8 @@ struct Barriers {
   uint64_t full[8];      // even CTA: a stage is complete in both CTAs
   uint64_t empty[8];
   uint64_t acc_full;
+  uint64_t acc_empty;    // even CTA: both CTAs' epilogues have read the accumulator
+  uint64_t drain;
   uint32_t tmem_base;
 };
 static_assert(sizeof(Barriers) <= kBarBytes, "barrier block");
@@ -148,12 +155,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1;
   const int n_tiles = (p.N + BN - 1) / BN;
-  const int m_cta = (pair / n_tiles) * (2 * BM) + (int)rank * BM;   // this CTA's A rows
-  const int n_pair = (pair % n_tiles) * BN;                          // pair's N columns
-  const int n_cta = n_pair + (int)rank * BNH;                        // this CTA's B rows
+  const int total_tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * n_tiles;
+  const int pair0 = blockIdx.x >> 1;
+  const int pair_stride = gridDim.x >> 1;
+  const int my_tiles = pair0 < total_tiles ? (total_tiles - pair0 + pair_stride - 1) / pair_stride : 0;
   const int nk = p.K / BK;
+  // tile i of this pair (i < my_tiles): rows and columns
+  auto tile_m = [&](int i) { return ((pair0 + i * pair_stride) / n_tiles) * (2 * BM) + (int)rank * BM; };
+  auto tile_n = [&](int i) { return ((pair0 + i * pair_stride) % n_tiles) * BN; };
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
@@ -167,6 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar->empty[s], 1);
       }
       mbar_init(&bar->acc_full, 1);
+      mbar_init(&bar->acc_empty, 16);  // 8 epilogue warps per CTA
+      mbar_init(&bar->drain, 1);
       fence_mbar_init();
     }
     __syncwarp();
@@ -177,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  const int total_kb = my_tiles * nk;
 
   if (warp == kTmaWarp) {
     // ---------------------------------------------------------------- TMA
@@ -185,94 +198,121 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kStageBytes = PACKED ? kPkStage : kI8Stage;
       constexpr int kABytes = PACKED ? kPkA : kI8A;
       constexpr int kColBytes = PACKED ? BK / 2 : BK;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % NS;
-        if (!mbar_wait(&bar->tma_empty[s], ((uint32_t)(kb / NS) & 1u) ^ 1u)) {
+      int i = 0, kb = 0, s = 0;
+      uint32_t ph = 0;
+      int row_a = my_tiles > 0 ? tile_m(0) : 0, row_b = my_tiles > 0 ? tile_n(0) + (int)rank * BNH : 0;
+      for (int g = 0; g < total_kb; ++g) {
+        if (!mbar_wait(&bar->tma_empty[s], ph ^ 1u)) {
           set_device_error(prm.err, kDevErrTimeoutEmpty);
           break;
         }
         const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
         mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
-        tma_load_2d(dst, &tmA, kb * kColBytes, m_cta, &bar->tma_full[s]);
-        tma_load_2d(dst + kABytes, &tmB, kb * kColBytes, n_cta, &bar->tma_full[s]);
+        tma_load_2d(dst, &tmA, kb * kColBytes, row_a, &bar->tma_full[s]);
+        tma_load_2d(dst + kABytes, &tmB, kb * kColBytes, row_b, &bar->tma_full[s]);
+        if (++s == NS) { s = 0; ph ^= 1u; }
+        if (++kb == nk) {
+          kb = 0;
+          if (++i < my_tiles) { row_a = tile_m(i); row_b = tile_n(i) + (int)rank * BNH; }
+        }
       }
     }
   } else if (warp == kMmaWarp) {
     if (!PACKED && !leader && lane == 0) {
       // relay: tell the even CTA when this CTA's operand tiles have landed
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S8;
-        if (!mbar_wait(&bar->tma_full[s], (uint32_t)(kb / S8) & 1u)) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int g = 0; g < total_kb; ++g) {
+        if (!mbar_wait(&bar->tma_full[s], ph)) {
           set_device_error(prm.err, kDevErrTimeoutFull);
           break;
         }
         mbar_arrive_remote(&bar->full[s], 0);
+        if (++s == S8) { s = 0; ph ^= 1u; }
       }
     }
     if (leader && lane == 0) {
       // ---------------------------------------------------------------- MMA
       constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
+      constexpr int NS = PACKED ? US : S8;
+      int s = 0;
+      uint32_t ph = 0;
       bool ok = true;
-      for (int kb = 0; kb < nk && ok; ++kb) {
-        if (PACKED) {
-          const int u = kb % US;
-          if (!mbar_wait(&bar->full[u], (uint32_t)(kb / US) & 1u)) {
-            set_device_error(prm.err, kDevErrTimeoutFull);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t b_stage = sbase + (uint32_t)(kPkRingBytes + u * kWideB);
-#pragma unroll
-          for (int ks = 0; ks < BK / 32; ++ks)
-            mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(u * (BK / 4) + ks * 8),
-                           smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc, (kb | ks) != 0 ? 1u : 0u);
-          tc_commit_pair_mc(&bar->empty[u], 0x3);
-        } else {
-          const int s = kb % S8;
-          const uint32_t ph = (uint32_t)(kb / S8) & 1u;
-          if (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait(&bar->full[s], ph)) {
-            set_device_error(prm.err, kDevErrTimeoutFull);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_stage = sbase + (uint32_t)(s * kI8Stage);
-#pragma unroll
-          for (int ks = 0; ks < BK / 32; ++ks)
-            mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
-                           smem_desc_kmajor_sw128(a_stage + kI8A + (uint32_t)(ks * 32)), idesc,
-                           (kb | ks) != 0 ? 1u : 0u);
-          tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        // the accumulator is free once both CTAs' epilogues have read tile i-1
+        if (i > 0 && !mbar_wait(&bar->acc_empty, (uint32_t)(i - 1) & 1u)) {
+          set_device_error(prm.err, kDevErrTimeoutAcc);
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb) {
+          if (PACKED) {
+            if (!mbar_wait(&bar->full[s], ph)) {
+              set_device_error(prm.err, kDevErrTimeoutFull);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t b_stage = sbase + (uint32_t)(kPkRingBytes + s * kWideB);
+#pragma unroll
+            for (int ks = 0; ks < BK / 32; ++ks)
+              mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8),
+                             smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
+                             (kb | ks) != 0 ? 1u : 0u);
+            tc_commit_pair_mc(&bar->empty[s], 0x3);
+          } else {
+            if (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait(&bar->full[s], ph)) {
+              set_device_error(prm.err, kDevErrTimeoutFull);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_stage = sbase + (uint32_t)(s * kI8Stage);
+#pragma unroll
+            for (int ks = 0; ks < BK / 32; ++ks)
+              mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
+                             smem_desc_kmajor_sw128(a_stage + kI8A + (uint32_t)(ks * 32)), idesc,
+                             (kb | ks) != 0 ? 1u : 0u);
+            tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
+          }
+          if (++s == NS) { s = 0; ph ^= 1u; }
+        }
+        tc_commit_pair_mc(&bar->acc_full, 0x3);
       }
-      tc_commit_pair_mc(&bar->acc_full, 0x3);
-      if (!mbar_wait(&bar->acc_full, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
+      // drain: every MMA issued so far has completed before teardown
+      tc_commit_pair_mc(&bar->drain, 0x1);
+      if (!mbar_wait(&bar->drain, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
     }
-  } else if (PACKED) {
-    // ---------------------------------------------------------------- widen
-    const bool is_a = warp < 4;
-    const int r = (warp & 3) * 32 + lane;                  // row within this CTA's tile
-    const uint32_t sw64 = (uint32_t)((r >> 1) & 3);
-    const uint32_t sw128 = (uint32_t)(r & 7);
-    const uint32_t a_taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + kACol0;
-    const uint32_t wide_row = sbase + (uint32_t)(kPkRingBytes + (r >> 3) * 1024 + (r & 7) * 128);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int ps = kb % PS;
-      const int u = kb % US;
-      if (!mbar_wait(&bar->tma_full[ps], (uint32_t)(kb / PS) & 1u)) {
+  } else if (warp < 8 || PACKED) {
+    // ------------------------------------------------ widen (INT4) + epilogue
+    // warps 0-7 widen A (TMEM) and run the epilogue; warps 8-15 widen B (smem).
+    // Two sets of warps take alternate k-blocks (set 0 even, set 1 odd) so
+    // that each warp has two MMA k-blocks of time per widen.
+    const bool is_a = warp < 8;
+    const int set = (warp >> 2) & 1;
+    const int quad = warp & 3;
+    const int half = set;                            // epilogue column half of an A warp
+    const int r = quad * 32 + lane;                   // operand row within this CTA's tile
+
+    // widen k-block g of this CTA's A or B rows
+    auto widen = [&](int g) -> bool {
+      const int ps = g % PS;
+      const int u = g % US;
+      if (!mbar_wait(&bar->tma_full[ps], (uint32_t)(g / PS) & 1u)) {
         set_device_error(prm.err, kDevErrTimeoutFull);
-        break;
+        return false;
       }
       const uint32_t src = sbase + (uint32_t)(ps * kPkStage + (is_a ? 0 : kPkA) + r * (BK / 2));
+      const uint32_t rsw64 = (uint32_t)((r >> 1) & 3);
       uint4 pk[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ sw64) << 4));
+      for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw64) << 4));
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->tma_empty[ps]);
-      if (!mbar_wait(&bar->empty[u], ((uint32_t)(kb / US) & 1u) ^ 1u)) {
+      if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
         set_device_error(prm.err, kDevErrTimeoutEmpty);
-        break;
+        return false;
       }
       tc_fence_after();
       if (is_a) {
@@ -284,107 +324,139 @@ __global__ void __launch_bounds__(kThreads, 1)
           regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
           regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
         }
-        tmem_st_32x32b_x32(a_taddr + (uint32_t)(u * (BK / 4)), regs);
+        tmem_st_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kACol0 + (uint32_t)(u * (BK / 4)), regs);
         tmem_wait_st();
         tc_fence_before();
       } else {
-        const uint32_t row = wide_row + (uint32_t)(u * kWideB);
+        const uint32_t row =
+            sbase + (uint32_t)(kPkRingBytes + u * kWideB + (r >> 3) * 1024 + (r & 7) * 128);
+        const uint32_t rsw128 = (uint32_t)(r & 7);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 c0, c1;
           widen16(pk[c], c0, c1);
-          st_shared_v4(row + ((((uint32_t)(2 * c)) ^ sw128) << 4), c0);
-          st_shared_v4(row + ((((uint32_t)(2 * c + 1)) ^ sw128) << 4), c1);
+          st_shared_v4(row + ((((uint32_t)(2 * c)) ^ rsw128) << 4), c0);
+          st_shared_v4(row + ((((uint32_t)(2 * c + 1)) ^ rsw128) << 4), c1);
         }
         fence_proxy_async_smem();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
-    }
-  }
+      return true;
+    };
 
-  // ------------------------------------------------------------ epilogue
-  if (warp < 8) {
-    const int quad = warp & 3;
-    const int half = warp >> 2;
+    // epilogue of tile i (A warps): dequant, low-rank, bias, bf16 TMA stores
     const uint32_t stage_out = sbase + (uint32_t)(ring_bytes<PACKED>() + warp * 2 * kStageTile);
-    float* s_sw = reinterpret_cast<float*>(smem_raw + (sbase - raw) + ring_bytes<PACKED>() + kOutStageBytes);
-    float* s_bias = s_sw + BN;
-    {
-      // this tile's weight scales and bias, staged once for all 256 threads
-      const int j = threadIdx.x;  // 0..255
-      const int n = n_pair + j;
-      s_sw[j] = n < p.N ? __ldg(p.b_scale + n) : 0.0f;
-      s_bias[j] = (p.bias && n < p.N) ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f;
-    }
-    named_barrier_sync(1, 256);
-    if (!mbar_wait(&bar->acc_full, 0)) set_device_error(prm.err, kDevErrTimeoutAcc);
-    tc_fence_after();
-    const int m_row0 = m_cta + quad * 32;
-    const long m = (long)m_row0 + lane;
-    const bool mok = m < p.M;
-    const float sa = mok ? __ldg(p.a_scale + m) : 0.0f;
+    float* vec_base = reinterpret_cast<float*>(smem_raw + (sbase - raw) + ring_bytes<PACKED>() + kOutStageBytes);
     const uint32_t sw64 = (uint32_t)((lane >> 1) & 3);
-#pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-      const int c0 = half * 128 + ch * 32;
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kAccCol + (uint32_t)c0, v);
-      tmem_wait_ld();
-      const int n = n_pair + c0;
-      if (n >= p.N) continue;  // warp-uniform
-      const int nv = min(32, p.N - n);
-      float y[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int acc = static_cast<int>(v[j]) >> kShift;
-        v[j] = static_cast<uint32_t>(acc);
-        y[j] = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa), s_sw[c0 + j]), p.inv_group);
+    int out_buf = 0;
+    auto epilogue = [&](int i) {
+      const int m_row0 = tile_m(i) + quad * 32;
+      const int n_pair = tile_n(i);
+      float* s_sw = vec_base + (i & 1) * 2 * BN;   // double-buffered by tile parity
+      float* s_bias = s_sw + BN;
+      {
+        const int j = threadIdx.x;  // 0..255
+        const int n = n_pair + j;
+        s_sw[j] = n < p.N ? __ldg(p.b_scale + n) : 0.0f;
+        s_bias[j] = (p.bias && n < p.N) ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f;
       }
-      if (p.rank > 0 && mok) {
-        const uint16_t* trow = p.T + m * p.rank;
+      named_barrier_sync(1, 256);
+      if (!mbar_wait(&bar->acc_full, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
+      tc_fence_after();
+      const long m = (long)m_row0 + lane;
+      const bool mok = m < p.M;
+      const float sa = mok ? __ldg(p.a_scale + m) : 0.0f;
 #pragma unroll 1
-        for (int jj = 0; jj < p.rank; ++jj) {
-          const float t = bf16_bits_to_float(trow[jj]);
-          const uint16_t* l2 = p.L2 + (long)jj * p.N + n;
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c0 = half * 128 + ch * 32;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kAccCol + (uint32_t)c0, v);
+        tmem_wait_ld();
+        if (ch == 3) {
+          // accumulator fully read by this warp: let the next tile's MMAs in
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(&bar->acc_empty, 0);
+        }
+        const int n = n_pair + c0;
+        if (n >= p.N) continue;  // warp-uniform
+        const int nv = min(32, p.N - n);
+        if (p.acc_debug && mok) {
+          uint4* dd = reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n);
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < nv) y[j] = __fmaf_rn(t, bf16_bits_to_float(__ldg(l2 + j)), y[j]);
+          for (int c = 0; c < 8; ++c)
+            if (4 * c < nv)
+              dd[c] = make_uint4((uint32_t)((int)v[4 * c] >> kShift), (uint32_t)((int)v[4 * c + 1] >> kShift),
+                                 (uint32_t)((int)v[4 * c + 2] >> kShift), (uint32_t)((int)v[4 * c + 3] >> kShift));
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int acc = static_cast<int>(v[j]) >> kShift;
+          v[j] = __float_as_uint(
+              __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa), s_sw[c0 + j]), p.inv_group));
+        }
+        if (p.rank > 0 && mok) {
+          const uint16_t* trow = p.T + m * p.rank;
+#pragma unroll 1
+          for (int jj = 0; jj < p.rank; ++jj) {
+            const float t = bf16_bits_to_float(trow[jj]);
+            const uint16_t* l2 = p.L2 + (long)jj * p.N + n;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nv) v[j] = __float_as_uint(__fmaf_rn(t, bf16_bits_to_float(__ldg(l2 + j)), __uint_as_float(v[j])));
+          }
+        }
+        uint32_t o[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float y0 = __fadd_rn(__uint_as_float(v[2 * j]), s_bias[c0 + 2 * j]);
+          const float y1 = __fadd_rn(__uint_as_float(v[2 * j + 1]), s_bias[c0 + 2 * j + 1]);
+          __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+          o[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        // stage the warp's 32 x 32 tile and let TMA write it (rows past M and
+        // columns past N are dropped by the tensor map bounds)
+        const uint32_t buf = stage_out + (uint32_t)(out_buf * kStageTile);
+        out_buf ^= 1;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(buf + (uint32_t)(lane * 64) + ((((uint32_t)c) ^ sw64) << 4),
+                       make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, buf, n, m_row0);
+          bulk_commit();
         }
       }
-      if (p.bias) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], s_bias[c0 + j]);
+    };
+
+    if (!PACKED) {
+      for (int i = 0; i < my_tiles; ++i) epilogue(i);
+    } else if (!is_a) {
+      for (int g = set; g < total_kb; g += 2)
+        if (!widen(g)) break;
+    } else {
+      // The epilogue of tile i-1 runs before this warp widens any k-block
+      // kb >= min(US, nk) of tile i: the first k-blocks of tile i are then
+      // ready the moment the accumulator is released, and nothing widened
+      // before the epilogue depends on tile i's MMAs.
+      const int lead = min(US, nk);
+      int next_epi = 0;
+      int i = 0, kb = set;
+      while (kb >= nk) { kb -= nk; ++i; }
+      for (int g = set; g < total_kb; g += 2) {
+        while (next_epi < i - 1 || (next_epi == i - 1 && kb >= lead)) epilogue(next_epi++);
+        if (!widen(g)) break;
+        kb += 2;
+        while (kb >= nk) { kb -= nk; ++i; }
       }
-      uint32_t o[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
-        o[j] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      // stage the warp's 32 x 32 tile and let TMA write it (rows past M and
-      // columns past N are dropped by the tensor map bounds)
-      const uint32_t buf = stage_out + (uint32_t)((ch & 1) * kStageTile);
-      if (lane == 0) bulk_wait_read<1>();
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        st_shared_v4(buf + (uint32_t)(lane * 64) + ((((uint32_t)c) ^ sw64) << 4),
-                     make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(&tmY, buf, n, m_row0);
-        bulk_commit();
-      }
-      if (p.acc_debug && mok) {
-        uint4* dd = reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          if (4 * c < nv) dd[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-      }
+      while (next_epi < my_tiles) epilogue(next_epi++);
     }
-    if (lane == 0) bulk_wait<0>();
+    if (is_a && lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
@@ -458,8 +530,15 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
       !make_tmap_bf16(&tY, a.Y, (uint64_t)a.M, (uint64_t)a.N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   const int pairs = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+  static int sm_count[64] = {0};
+  if (dev < 64 && !sm_count[dev]) {
+    int n = 0;
+    if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    sm_count[dev] = n;
+  }
+  const int sms = dev < 64 ? sm_count[dev] : 148;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.gridDim = dim3(2 * std::min(pairs, sms / 2), 1, 1);   // persistent: one pair per TPC
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes<PACKED>();
   cfg.stream = st;
