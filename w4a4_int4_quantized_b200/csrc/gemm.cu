@@ -83,7 +83,7 @@ constexpr uint32_t kTmemCols = 512;
 // stores (64-byte rows, 64-byte swizzle), then the tile's weight scales and
 // bias in fp32
 constexpr int kStageTile = 32 * 32 * 2;               // 2 KB
-constexpr int kOutStageBytes = 8 * 2 * kStageTile;     // 32 KB
+constexpr int kOutStageBytes = 16 * kStageTile;        // 32 KB: one tile per epilogue warp
 constexpr int kVecBytes = 2 * 2 * BN * 4;              // 4 KB (two tiles)
 constexpr int kBarBytes = 512;
 template <bool PACKED>
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar->empty[s], 1);
       }
       mbar_init(&bar->acc_full, 1);
-      mbar_init(&bar->acc_empty, 16);  // 8 epilogue warps per CTA
+      mbar_init(&bar->acc_empty, 32);  // 16 epilogue warps per CTA
       mbar_init(&bar->drain, 1);
       fence_mbar_init();
     }
@@ -190,6 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
   const int total_kb = my_tiles * nk;
+  // everything above overlaps the tail of the kernel producing the codes
+  grid_dependency_wait();
 
   if (warp == kTmaWarp) {
     // ---------------------------------------------------------------- TMA
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit_pair_mc(&bar->drain, 0x1);
       if (!mbar_wait(&bar->drain, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
     }
-  } else if (warp < 8 || PACKED) {
+  } else if (warp < 16) {
     // ------------------------------------------------ widen (INT4) + epilogue
     // warps 0-7 widen A (TMEM) and run the epilogue; warps 8-15 widen B (smem).
     // Two sets of warps take alternate k-blocks (set 0 even, set 1 odd) so
@@ -292,7 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool is_a = warp < 8;
     const int set = (warp >> 2) & 1;
     const int quad = warp & 3;
-    const int half = set;                            // epilogue column half of an A warp
     const int r = quad * 32 + lane;                   // operand row within this CTA's tile
 
     // widen k-block g of this CTA's A or B rows
@@ -345,55 +346,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    // epilogue of tile i (A warps): dequant, low-rank, bias, bf16 TMA stores
-    const uint32_t stage_out = sbase + (uint32_t)(ring_bytes<PACKED>() + warp * 2 * kStageTile);
+    // epilogue of tile i: each of the 16 warps drains 64 accumulator columns
+    // of its TMEM lane quadrant into registers, releases the accumulator to
+    // the next tile's MMAs, then dequantizes, adds the low-rank term and the
+    // bias and writes bf16 through TMA stores.
+    const int cq = warp >> 2;                         // column quarter (64 columns)
+    const uint32_t stage_out = sbase + (uint32_t)(ring_bytes<PACKED>() + warp * kStageTile);
     float* vec_base = reinterpret_cast<float*>(smem_raw + (sbase - raw) + ring_bytes<PACKED>() + kOutStageBytes);
     const uint32_t sw64 = (uint32_t)((lane >> 1) & 3);
-    int out_buf = 0;
     auto epilogue = [&](int i) {
       const int m_row0 = tile_m(i) + quad * 32;
       const int n_pair = tile_n(i);
       float* s_sw = vec_base + (i & 1) * 2 * BN;   // double-buffered by tile parity
       float* s_bias = s_sw + BN;
-      {
-        const int j = threadIdx.x;  // 0..255
+      if (threadIdx.x < BN) {
+        const int j = threadIdx.x;
         const int n = n_pair + j;
         s_sw[j] = n < p.N ? __ldg(p.b_scale + n) : 0.0f;
         s_bias[j] = (p.bias && n < p.N) ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f;
       }
-      named_barrier_sync(1, 256);
-      if (!mbar_wait(&bar->acc_full, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
-      tc_fence_after();
+      named_barrier_sync(1, 512);
       const long m = (long)m_row0 + lane;
       const bool mok = m < p.M;
       const float sa = mok ? __ldg(p.a_scale + m) : 0.0f;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        const int c0 = half * 128 + ch * 32;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kAccCol + (uint32_t)c0, v);
-        tmem_wait_ld();
-        if (ch == 3) {
-          // accumulator fully read by this warp: let the next tile's MMAs in
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(&bar->acc_empty, 0);
-        }
+      if (!mbar_wait(&bar->acc_full, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
+      tc_fence_after();
+      uint32_t v[2][32];
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + kAccCol + (uint32_t)(cq * 64);
+      tmem_ld_32x32b_x32(taddr, v[0]);
+      tmem_ld_32x32b_x32(taddr + 32, v[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(&bar->acc_empty, 0);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int c0 = cq * 64 + ch * 32;
         const int n = n_pair + c0;
         if (n >= p.N) continue;  // warp-uniform
         const int nv = min(32, p.N - n);
+        uint32_t* vv = v[ch];
         if (p.acc_debug && mok) {
           uint4* dd = reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             if (4 * c < nv)
-              dd[c] = make_uint4((uint32_t)((int)v[4 * c] >> kShift), (uint32_t)((int)v[4 * c + 1] >> kShift),
-                                 (uint32_t)((int)v[4 * c + 2] >> kShift), (uint32_t)((int)v[4 * c + 3] >> kShift));
+              dd[c] = make_uint4((uint32_t)((int)vv[4 * c] >> kShift), (uint32_t)((int)vv[4 * c + 1] >> kShift),
+                                 (uint32_t)((int)vv[4 * c + 2] >> kShift), (uint32_t)((int)vv[4 * c + 3] >> kShift));
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int acc = static_cast<int>(v[j]) >> kShift;
-          v[j] = __float_as_uint(
+          const int acc = static_cast<int>(vv[j]) >> kShift;
+          vv[j] = __float_as_uint(
               __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa), s_sw[c0 + j]), p.inv_group));
         }
         if (p.rank > 0 && mok) {
@@ -404,31 +408,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint16_t* l2 = p.L2 + (long)jj * p.N + n;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < nv) v[j] = __float_as_uint(__fmaf_rn(t, bf16_bits_to_float(__ldg(l2 + j)), __uint_as_float(v[j])));
+              if (j < nv)
+                vv[j] = __float_as_uint(__fmaf_rn(t, bf16_bits_to_float(__ldg(l2 + j)), __uint_as_float(vv[j])));
           }
         }
         uint32_t o[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float y0 = __fadd_rn(__uint_as_float(v[2 * j]), s_bias[c0 + 2 * j]);
-          const float y1 = __fadd_rn(__uint_as_float(v[2 * j + 1]), s_bias[c0 + 2 * j + 1]);
+          const float y0 = __fadd_rn(__uint_as_float(vv[2 * j]), s_bias[c0 + 2 * j]);
+          const float y1 = __fadd_rn(__uint_as_float(vv[2 * j + 1]), s_bias[c0 + 2 * j + 1]);
           __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
           o[j] = *reinterpret_cast<uint32_t*>(&h);
         }
         // stage the warp's 32 x 32 tile and let TMA write it (rows past M and
         // columns past N are dropped by the tensor map bounds)
-        const uint32_t buf = stage_out + (uint32_t)(out_buf * kStageTile);
-        out_buf ^= 1;
-        if (lane == 0) bulk_wait_read<1>();
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          st_shared_v4(buf + (uint32_t)(lane * 64) + ((((uint32_t)c) ^ sw64) << 4),
+          st_shared_v4(stage_out + (uint32_t)(lane * 64) + ((((uint32_t)c) ^ sw64) << 4),
                        make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmY, buf, n, m_row0);
+          tma_store_2d(&tmY, stage_out, n, m_row0);
           bulk_commit();
         }
       }
@@ -436,9 +439,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (!PACKED) {
       for (int i = 0; i < my_tiles; ++i) epilogue(i);
-    } else if (!is_a) {
-      for (int g = set; g < total_kb; g += 2)
-        if (!widen(g)) break;
     } else {
       // The epilogue of tile i-1 runs before this warp widens any k-block
       // kb >= min(US, nk) of tile i: the first k-blocks of tile i are then
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       while (next_epi < my_tiles) epilogue(next_epi++);
     }
-    if (is_a && lane == 0) bulk_wait<0>();
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
@@ -542,13 +542,15 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes<PACKED>();
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   Params prm{a, err};
   e = cudaLaunchKernelEx(&cfg, gemm_kernel<PACKED>, prm, tA, tB, tY);
   if (e != cudaSuccess) return e;

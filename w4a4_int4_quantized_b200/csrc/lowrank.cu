@@ -11,6 +11,7 @@
 // slabs of L1.  Rank r <= 256 keeps this a thin product (2 M K r flops).
 #include <cuda_bf16.h>
 
+#include "common.cuh"
 #include "kernels.h"
 
 namespace w4a4 {
@@ -26,6 +27,7 @@ __global__ void __launch_bounds__(256) lowrank_down_kernel(const uint16_t* __res
                                                            uint16_t* __restrict__ T) {
   __shared__ float xs[TK][TM + 1];
   __shared__ float ls[TK][TN + 1];
+  grid_launch_dependents();
   const int m0 = blockIdx.y * TM, j0 = blockIdx.x * TN;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   float acc[4][4] = {};

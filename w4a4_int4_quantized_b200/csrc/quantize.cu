@@ -143,6 +143,10 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
   };
 
   rowmax[0][tid] = 0u;
+  // launched with programmatic stream serialization: wait for the previous
+  // kernel of the stream (it may produce X, or still read this output)
+  grid_dependency_wait();
+  grid_launch_dependents();
 #pragma unroll
   for (int it = 0; it < kStages - 1; ++it) issue(it);
 
@@ -177,7 +181,10 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
         }
       }
       if (ROT) {
-        // stages h = 1 .. HALF/2: pairs (i, i+h) sit in different float2s
+        // stages h = 1 .. HALF/2: pairs (i, i+h) sit in different float2s.
+        // a - b is formed as fma(b, -1, a): the product is exact, so this is
+        // the single IEEE subtraction, without a separate negation.
+        const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
         for (int h = 1; h < HALF; h <<= 1) {
 #pragma unroll
@@ -185,21 +192,29 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
             if ((i & h) == 0) {
               const float2 a = P[i], b = P[i + h];
               P[i] = __fadd2_rn(a, b);
-              P[i + h] = __fadd2_rn(a, make_float2(-b.x, -b.y));
+              P[i + h] = __ffma2_rn(b, m1, a);
             }
           }
         }
-        // last stage h = HALF: the two halves of each float2
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const float a = P[i].x, b = P[i].y;
-          P[i].x = __fadd_rn(a, b);
-          P[i].y = __fsub_rn(a, b);
-        }
       }
       float amax = 0.0f;
+      if (ROT) {
+        // last stage h = HALF on the two halves of each float2.  Its outputs
+        // a + b and a - b have max(|a + b|, |a - b|) = fl(|a| + |b|) exactly
+        // (rounding is monotone and sign-symmetric), which gives the absmax.
 #pragma unroll
-      for (int i = 0; i < HALF; ++i) amax = max3(amax, fabsf(P[i].x), fabsf(P[i].y));
+        for (int i = 0; i < HALF; i += 2) {
+          const float a0 = P[i].x, b0 = P[i].y, a1 = P[i + 1].x, b1 = P[i + 1].y;
+          amax = max3(amax, __fadd_rn(fabsf(a0), fabsf(b0)), __fadd_rn(fabsf(a1), fabsf(b1)));
+          P[i].x = __fadd_rn(a0, b0);
+          P[i].y = __fsub_rn(a0, b0);
+          P[i + 1].x = __fadd_rn(a1, b1);
+          P[i + 1].y = __fsub_rn(a1, b1);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) amax = max3(amax, fabsf(P[i].x), fabsf(P[i].y));
+      }
       atomicMax(&rmax[lr], __float_as_uint(amax));
     }
     __syncthreads();
@@ -270,11 +285,35 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
     if (e != cudaSuccess) return e;
     attr_set[dev] = smem;
   }
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess) return e;
+  // occupancy of the last K seen on each device (deterministic, so a racing
+  // refresh only repeats the query)
+  static int cache_k[64] = {0}, cache_sms[64] = {0}, cache_per_sm[64] = {0};
+  if (dev < 64 && cache_k[dev] == K) {
+    sms = cache_sms[dev];
+    per_sm = cache_per_sm[dev];
+  } else {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess) return e;
+    if (dev < 64) {
+      cache_sms[dev] = sms;
+      cache_per_sm[dev] = per_sm;
+      cache_k[dev] = K;
+    }
+  }
   const int nblk = (M + rows_per_blk - 1) / rows_per_blk;
   const int grid = min(nblk, sms * max(per_sm, 1));
-  kern<<<grid, threads, smem, st>>>(X, M, K, rows_per_blk, out, scale);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, rows_per_blk, out, scale);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
