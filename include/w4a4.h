@@ -138,6 +138,28 @@ w4a4_status w4a4_linear(const void* X, const uint8_t* Wq, const float* w_scale, 
                         const void* L1, const void* L2, int rank, const void* bias, void* Y, void* workspace,
                         size_t workspace_bytes, w4a4_stream_t stream);
 
+/* Allocation-free form of w4a4_linear.  The pages have no counterpart: this
+ * serves callers that cannot allocate device memory -- for instance a host
+ * program that has given all device memory to its own fixed pool, or a plugin
+ * running inside a runtime that forbids cudaMalloc after start-up -- and so
+ * cannot pass the workspace w4a4_linear needs.
+ *   Scratch: a fixed array of W4A4_NOALLOC_SCRATCH_BYTES inside the library,
+ *     one per GPU that loads the library, kept until the process exits.  The
+ *     call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine).  Layers whose w4a4_workspace_bytes(M, K, rank) exceeds the
+ *     scratch are rejected with W4A4_ERR_WORKSPACE; use w4a4_linear for them.
+ *   The first call on a device looks up the scratch address on that device
+ *     (with it current); make that first call before any stream capture.
+ *   All calls share the scratch.  Calls that may overlap on the GPU (other
+ *     streams, other host threads) race on it and must be serialised by the
+ *     caller.  The scratch keeps the last call's contents; every byte a call
+ *     reads is written earlier in the same call, so nothing is cleared.
+ *   Arguments, results and errors are otherwise those of w4a4_linear. */
+#define W4A4_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+w4a4_status w4a4_linear_noalloc(const void* X, const uint8_t* Wq, const float* w_scale, int M, int N, int K,
+                                int group, const void* L1, const void* L2, int rank, const void* bias, void* Y,
+                                w4a4_stream_t stream);
+
 /* ---------------------------------------------------------------- W8A8 */
 /* The INT8 path for sensitive layers ("ComfyUI-INT4-Fast" (kongchang.com),
  * "Per-Layer Dynamic Routing"; "W4A4 and W4A8" (renderbob.io), "How the

@@ -19,7 +19,7 @@ __all__ = [
     "W4A4Error", "library_path", "load_library",
     "w4a4_version", "w4a4_status_string",
     "w4a4_quantize_weights", "w4a4_rotate_quantize_act", "w4a4_gemm", "w4a4_linear",
-    "w4a4_workspace_bytes",
+    "w4a4_workspace_bytes", "w4a4_linear_noalloc", "NOALLOC_SCRATCH_BYTES",
     "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
     "w8a8_workspace_bytes", "w4a4_get_device_error",
 ]
@@ -63,6 +63,7 @@ def load_library():
         "w4a4_gemm": ([P, P, P, P, I, I, I, I, P, P, I, P, P, P, P], S),
         "w4a4_workspace_bytes": ([I, I, I], Z),
         "w4a4_linear": ([P, P, P, I, I, I, I, P, P, I, P, P, P, Z, P], S),
+        "w4a4_linear_noalloc": ([P, P, P, I, I, I, I, P, P, I, P, P, P], S),
         "w8a8_quantize_weights": ([P, I, I, I, P, P, P], S),
         "w8a8_rotate_quantize_act": ([P, I, I, I, P, P, P], S),
         "w8a8_gemm": ([P, P, P, P, I, I, I, I, P, P, P, P], S),
@@ -161,6 +162,24 @@ def w4a4_linear(X, Wq, w_scale, group, L1=None, L2=None, bias=None, Y=None, work
     _check("w4a4_linear", load_library().w4a4_linear(
         _ptr(X), _ptr(Wq), _ptr(w_scale), M, N, K, group, _ptr(L1), _ptr(L2), rank, _ptr(bias), _ptr(Y),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return Y
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024   # W4A4_NOALLOC_SCRATCH_BYTES in include/w4a4.h
+
+
+def w4a4_linear_noalloc(X, Wq, w_scale, group, L1=None, L2=None, bias=None, Y=None, stream=None):
+    """w4a4_linear on the library's built-in scratch: the C call allocates no
+    device memory (Y is allocated here with torch only when not passed in).
+    Layers needing more than NOALLOC_SCRATCH_BYTES of scratch are rejected."""
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    rank = 0 if L1 is None else L1.shape[1]
+    Y = _empty((M, N), torch.bfloat16, X) if Y is None else Y
+    _check("w4a4_linear_noalloc", load_library().w4a4_linear_noalloc(
+        _ptr(X), _ptr(Wq), _ptr(w_scale), M, N, K, group, _ptr(L1), _ptr(L2), rank, _ptr(bias), _ptr(Y),
+        _stream(stream)))
     return Y
 
 
