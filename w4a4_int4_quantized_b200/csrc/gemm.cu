@@ -19,22 +19,28 @@
 // shift of the int32 accumulator (|acc| <= 64 K << 2^23 for K <= 32768).
 //
 // Work decomposition: a cluster of two CTAs (one per SM of a TPC) owns a
-// 256 x 256 output tile and issues the pair form of the MMA (cta_group::2):
-// each CTA holds 128 rows of A, 128 rows (N) of B and its 128 x 256 int32
+// 256 x BN output tile and issues the pair form of the MMA (cta_group::2):
+// each CTA holds 128 rows of A, BN/2 rows (N) of B and its 128 x BN int32
 // accumulator.  Per CTA (k-block = 128 codes):
-//   warp 8      TMA: packed A and B tiles (64-byte rows, 64-byte swizzle)
-//               into a 6-deep shared-memory ring (no multicast);
-//   warps 0-3   widen A rows (one row per thread, conflict-free 16-byte
-//               reads) and tcgen05.st them into a 4-deep TMEM ring -- A is
-//               read by the MMA from tensor memory;
-//   warps 4-7   widen B rows into a 4-deep ring in the 128-byte-swizzled
-//               K-major layout the MMA reads from shared memory;
-//   warp 9      (even CTA) one thread issues the pair MMAs and commits each
-//               stage to the barriers of both CTAs.
-//   warps 0-7   epilogue: tcgen05.ld, dequant, low-rank, bias, bf16 stores.
+//   warp 16     TMA: packed A and B tiles (64-byte rows, 64-byte swizzle)
+//               into a shared-memory ring (no multicast), and per tile the
+//               low-rank operand tiles T and L2;
+//   warps 0-7   widen A rows (one row per thread, conflict-free 16-byte
+//               reads) and tcgen05.st them into a TMEM ring -- A is read by
+//               the MMA from tensor memory;
+//   warps 8-15  widen B rows into a ring in the 128-byte-swizzled K-major
+//               layout the MMA reads from shared memory;
+//               (two sets of warps take alternate k-blocks)
+//   warp 17     (even CTA) one thread issues the pair MMAs and commits each
+//               stage to the barriers of both CTAs; (odd CTA) relays the
+//               arrival of TMA-only operands to the even CTA.
+//   warps 0-15  epilogue: tcgen05.ld, dequant, low-rank, bias, bf16 TMA
+//               stores.
 // The kernel is persistent: one pair per TPC walks its output tiles, and the
 // TMA and widen stages run ahead into the next tile while the epilogue of the
-// current one drains the (single) accumulator.
+// current one drains the accumulator.  With a low-rank branch the tile is
+// 256 x 128, so that TMEM holds the int32 accumulator, an fp32 accumulator
+// for T L2 (bf16 MMAs issued after each tile's integer MMAs) and the A ring.
 // The INT8 path skips the widening: TMA writes both operands straight into
 // the 128-byte-swizzled layout and the MMA reads both from shared memory.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
@@ -53,48 +59,48 @@ namespace w4a4 {
 namespace {
 
 constexpr int BM = 128;          // A rows per CTA; the pair covers 256
-constexpr int BN = 256;          // N per pair tile
-constexpr int BNH = BN / 2;      // B rows staged per CTA
 constexpr int BK = 128;          // codes per k-block
 constexpr int kThreads = 576;    // 18 warps
 constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
-
-// packed (INT4) path
-constexpr int PS = 5;                                // packed TMA stages
-constexpr int US = 6;                                // widened stages
-constexpr int kPkA = BM * BK / 2;                    // 8 KB
-constexpr int kPkB = BNH * BK / 2;                   // 8 KB
-constexpr int kPkStage = kPkA + kPkB;
-constexpr int kWideB = BNH * BK;                     // 16 KB
-constexpr int kPkRingBytes = PS * kPkStage;          // 80 KB
-constexpr int kWideRingBytes = US * kWideB;          // 96 KB
-// int8 path
-constexpr int S8 = 5;
-constexpr int kI8A = BM * BK;                        // 16 KB
-constexpr int kI8B = BNH * BK;                       // 16 KB
-constexpr int kI8Stage = kI8A + kI8B;
-
-constexpr uint32_t kAccCol = 0;                      // int32 accumulator: columns [0, 256)
-constexpr uint32_t kACol0 = 256;                     // A ring: 32 columns per stage
+constexpr int PS = 5;            // packed TMA stages
+constexpr int US = 6;            // widened stages
+constexpr int S8 = 5;            // INT8 TMA stages
+constexpr int LRC = 128;         // low-rank rank chunk per MMA round
 constexpr uint32_t kTmemCols = 512;
-
-// epilogue: per-warp double-buffered 32 x 32 bf16 staging tiles for TMA
-// stores (64-byte rows, 64-byte swizzle), then the tile's weight scales and
-// bias in fp32
-constexpr int kStageTile = 32 * 32 * 2;               // 2 KB
-constexpr int kOutStageBytes = 16 * kStageTile;        // 32 KB: one tile per epilogue warp
-constexpr int kVecBytes = 2 * 2 * BN * 4;              // 4 KB (two tiles)
+constexpr uint32_t kAccCol = 0;  // int32 accumulator
+constexpr uint32_t kACol0 = 256; // A ring: 32 columns per stage
+constexpr int kStageTile = 32 * 32 * 2;            // epilogue staging tile: 32 x 32 bf16
+constexpr int kOutStageBytes = 16 * kStageTile;    // one per epilogue warp
 constexpr int kBarBytes = 512;
-template <bool PACKED>
-constexpr int ring_bytes() { return PACKED ? kPkRingBytes + kWideRingBytes : S8 * kI8Stage; }
-template <bool PACKED>
-constexpr int data_bytes() { return ring_bytes<PACKED>() + kOutStageBytes + kVecBytes; }
-template <bool PACKED>
-constexpr int smem_bytes() { return data_bytes<PACKED>() + kBarBytes + 1024; }
-static_assert(smem_bytes<true>() <= 232448 && smem_bytes<false>() <= 232448, "shared memory budget");
 
-static_assert(kACol0 + US * (BK / 4) <= kTmemCols, "TMEM budget");
+template <bool PACKED, bool LR>
+struct Cfg {
+  static constexpr int BN = LR ? 128 : 256;          // N per pair tile
+  static constexpr int BNH = BN / 2;                 // B rows staged per CTA
+  static constexpr int kPkA = BM * BK / 2;           // packed A stage (8 KB)
+  static constexpr int kPkB = BNH * BK / 2;
+  static constexpr int kPkStage = kPkA + kPkB;
+  static constexpr int kWideB = BNH * BK;            // widened B stage
+  static constexpr int kI8A = BM * BK;               // INT8 stages
+  static constexpr int kI8B = BNH * BK;
+  static constexpr int kI8Stage = kI8A + kI8B;
+  static constexpr int kRing = PACKED ? PS * kPkStage + US * kWideB : S8 * kI8Stage;
+  static constexpr int kLrT = BM * LRC * 2;          // T chunk: 128 rows x 128 ranks, two 64-wide boxes
+  static constexpr int kLrL2 = BNH * LRC * 2;        // L2 chunk: 128 ranks x BNH columns
+  static constexpr int kLrBytes = LR ? kLrT + kLrL2 : 0;
+  static constexpr int kVecBytes = 2 * 2 * BN * 4;   // scales + bias, two tiles
+  static constexpr int kLrOff = kRing;
+  static constexpr int kOutOff = kLrOff + kLrBytes;
+  static constexpr int kVecOff = kOutOff + kOutStageBytes;
+  static constexpr int kDataBytes = kVecOff + kVecBytes;
+  static constexpr int kSmemBytes = kDataBytes + kBarBytes + 1024;
+  static constexpr uint32_t kLrCol = BN;             // fp32 low-rank accumulator (LR only)
+  static constexpr int kColsPerWarp = BN / 4;        // epilogue: 4 warps per TMEM lane quadrant
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kACol0 + US * (BK / 4) <= kTmemCols, "TMEM budget");
+  static_assert(!LR || kLrCol + BN <= kACol0, "TMEM budget (low-rank accumulator)");
+};
 
 struct Params {
   GemmArgs a;
@@ -106,8 +112,11 @@ struct Barriers {
   uint64_t tma_empty[8];
   uint64_t full[8];      // even CTA: a stage is complete in both CTAs
   uint64_t empty[8];
+  uint64_t lr_full;      // this CTA's low-rank chunk landed (TMA)
+  uint64_t lr_ready;     // even CTA: the odd CTA's low-rank chunk landed (relay)
+  uint64_t lr_empty;     // the low-rank MMAs of the chunk completed
   uint64_t acc_full;
-  uint64_t acc_empty;    // even CTA: both CTAs' epilogues have read the accumulator
+  uint64_t acc_empty;    // even CTA: both CTAs' epilogues have read the accumulators
   uint64_t drain;
   uint32_t tmem_base;
 };
@@ -140,16 +149,20 @@ __device__ __forceinline__ void widen16(const uint4 p, uint4& c0, uint4& c1) {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-template <bool PACKED>
+template <bool PACKED, bool LR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmY) {
+                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
+                const __grid_constant__ CUtensorMap tmL2) {
+  using C = Cfg<PACKED, LR>;
+  constexpr int BN = C::BN;
+  constexpr int BNH = C::BNH;
   const GemmArgs& p = prm.a;
   constexpr int kShift = PACKED ? 8 : 0;  // widened products carry 2^8
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  Barriers* bar = reinterpret_cast<Barriers*>(smem_raw + (sbase - raw) + data_bytes<PACKED>());
+  Barriers* bar = reinterpret_cast<Barriers*>(smem_raw + (sbase - raw) + C::kDataBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -161,7 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair_stride = gridDim.x >> 1;
   const int my_tiles = pair0 < total_tiles ? (total_tiles - pair0 + pair_stride - 1) / pair_stride : 0;
   const int nk = p.K / BK;
-  // tile i of this pair (i < my_tiles): rows and columns
+  const int lr_chunks = LR ? (p.rank + LRC - 1) / LRC : 0;
+  // tile i of this pair (i < my_tiles): this CTA's rows, the pair's columns
   auto tile_m = [&](int i) { return ((pair0 + i * pair_stride) / n_tiles) * (2 * BM) + (int)rank * BM; };
   auto tile_n = [&](int i) { return ((pair0 + i * pair_stride) % n_tiles) * BN; };
 
@@ -170,12 +184,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
       prefetch_tmap(&tmY);
+      if (LR) {
+        prefetch_tmap(&tmT);
+        prefetch_tmap(&tmL2);
+      }
       for (int s = 0; s < 8; ++s) {
         mbar_init(&bar->tma_full[s], 1);
         mbar_init(&bar->tma_empty[s], PACKED ? 8 : 1);
         mbar_init(&bar->full[s], PACKED ? 16 : 1);  // 8 widen warps per CTA, or 1 relay
         mbar_init(&bar->empty[s], 1);
       }
+      mbar_init(&bar->lr_full, 1);
+      mbar_init(&bar->lr_ready, 1);
+      mbar_init(&bar->lr_empty, 1);
       mbar_init(&bar->acc_full, 1);
       mbar_init(&bar->acc_empty, 32);  // 16 epilogue warps per CTA
       mbar_init(&bar->drain, 1);
@@ -197,51 +218,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       constexpr int NS = PACKED ? PS : S8;
-      constexpr int kStageBytes = PACKED ? kPkStage : kI8Stage;
-      constexpr int kABytes = PACKED ? kPkA : kI8A;
+      constexpr int kStageBytes = PACKED ? C::kPkStage : C::kI8Stage;
+      constexpr int kABytes = PACKED ? C::kPkA : C::kI8A;
       constexpr int kColBytes = PACKED ? BK / 2 : BK;
-      int i = 0, kb = 0, s = 0;
+      int s = 0, lr_n = 0;
       uint32_t ph = 0;
-      int row_a = my_tiles > 0 ? tile_m(0) : 0, row_b = my_tiles > 0 ? tile_n(0) + (int)rank * BNH : 0;
-      for (int g = 0; g < total_kb; ++g) {
-        if (!mbar_wait(&bar->tma_empty[s], ph ^ 1u)) {
-          set_device_error(prm.err, kDevErrTimeoutEmpty);
-          break;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int row_a = tile_m(i);
+        const int row_b = tile_n(i) + (int)rank * BNH;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&bar->tma_empty[s], ph ^ 1u)) {
+            set_device_error(prm.err, kDevErrTimeoutEmpty);
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
+          mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
+          tma_load_2d(dst, &tmA, kb * kColBytes, row_a, &bar->tma_full[s]);
+          tma_load_2d(dst + kABytes, &tmB, kb * kColBytes, row_b, &bar->tma_full[s]);
+          if (++s == NS) { s = 0; ph ^= 1u; }
         }
-        const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
-        mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
-        tma_load_2d(dst, &tmA, kb * kColBytes, row_a, &bar->tma_full[s]);
-        tma_load_2d(dst + kABytes, &tmB, kb * kColBytes, row_b, &bar->tma_full[s]);
-        if (++s == NS) { s = 0; ph ^= 1u; }
-        if (++kb == nk) {
-          kb = 0;
-          if (++i < my_tiles) { row_a = tile_m(i); row_b = tile_n(i) + (int)rank * BNH; }
+        if (LR) {
+          // low-rank operand chunks of this tile: T rows (K-major, two
+          // 64-rank boxes) and L2 columns (N-major, one 128-rank box)
+          for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
+            if (!mbar_wait(&bar->lr_empty, ((uint32_t)lr_n & 1u) ^ 1u)) {
+              set_device_error(prm.err, kDevErrTimeoutEmpty);
+              ok = false;
+              break;
+            }
+            const uint32_t lr = sbase + (uint32_t)C::kLrOff;
+            const bool second = p.rank - c * LRC > 64;   // ranks past 64 in this chunk
+            mbar_arrive_expect_tx(&bar->lr_full, (uint32_t)((second ? C::kLrT : C::kLrT / 2) + C::kLrL2));
+            tma_load_2d(lr, &tmT, c * LRC, row_a, &bar->lr_full);
+            if (second) tma_load_2d(lr + C::kLrT / 2, &tmT, c * LRC + 64, row_a, &bar->lr_full);
+            tma_load_2d(lr + C::kLrT, &tmL2, row_b, c * LRC, &bar->lr_full);
+          }
         }
       }
     }
   } else if (warp == kMmaWarp) {
-    if (!PACKED && !leader && lane == 0) {
-      // relay: tell the even CTA when this CTA's operand tiles have landed
-      int s = 0;
+    if (!leader && lane == 0) {
+      // relay: tell the even CTA when this CTA's TMA-only operands have landed
+      int s = 0, lr_n = 0;
       uint32_t ph = 0;
-      for (int g = 0; g < total_kb; ++g) {
-        if (!mbar_wait(&bar->tma_full[s], ph)) {
-          set_device_error(prm.err, kDevErrTimeoutFull);
-          break;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        if (!PACKED) {
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait(&bar->tma_full[s], ph)) {
+              set_device_error(prm.err, kDevErrTimeoutFull);
+              ok = false;
+              break;
+            }
+            mbar_arrive_remote(&bar->full[s], 0);
+            if (++s == S8) { s = 0; ph ^= 1u; }
+          }
         }
-        mbar_arrive_remote(&bar->full[s], 0);
-        if (++s == S8) { s = 0; ph ^= 1u; }
+        for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
+          if (!mbar_wait(&bar->lr_full, (uint32_t)lr_n & 1u)) {
+            set_device_error(prm.err, kDevErrTimeoutFull);
+            ok = false;
+            break;
+          }
+          mbar_arrive_remote(&bar->lr_ready, 0);
+        }
       }
     }
     if (leader && lane == 0) {
       // ---------------------------------------------------------------- MMA
       constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
+      constexpr uint32_t idesc_lr = idesc_bf16(2 * BM, BN, false, true);
       constexpr int NS = PACKED ? US : S8;
-      int s = 0;
+      int s = 0, lr_n = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
-        // the accumulator is free once both CTAs' epilogues have read tile i-1
+        // the accumulators are free once both CTAs' epilogues have read tile i-1
         if (i > 0 && !mbar_wait(&bar->acc_empty, (uint32_t)(i - 1) & 1u)) {
           set_device_error(prm.err, kDevErrTimeoutAcc);
           ok = false;
@@ -256,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t b_stage = sbase + (uint32_t)(kPkRingBytes + s * kWideB);
+            const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
 #pragma unroll
             for (int ks = 0; ks < BK / 32; ++ks)
               mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8),
@@ -270,15 +324,37 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a_stage = sbase + (uint32_t)(s * kI8Stage);
+            const uint32_t a_stage = sbase + (uint32_t)(s * C::kI8Stage);
 #pragma unroll
             for (int ks = 0; ks < BK / 32; ++ks)
               mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
-                             smem_desc_kmajor_sw128(a_stage + kI8A + (uint32_t)(ks * 32)), idesc,
+                             smem_desc_kmajor_sw128(a_stage + C::kI8A + (uint32_t)(ks * 32)), idesc,
                              (kb | ks) != 0 ? 1u : 0u);
             tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
           }
           if (++s == NS) { s = 0; ph ^= 1u; }
+        }
+        if (LR) {
+          // T L2 into the fp32 accumulator: A = T (K-major, 128-byte
+          // swizzle, k-step 16 ranks = 32 bytes), B = L2 (N-major, 128-byte
+          // swizzle, k-step 16 ranks = two 8-row atoms)
+          for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
+            if (!mbar_wait(&bar->lr_full, (uint32_t)lr_n & 1u) || !mbar_wait(&bar->lr_ready, (uint32_t)lr_n & 1u)) {
+              set_device_error(prm.err, kDevErrTimeoutFull);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t lr = sbase + (uint32_t)C::kLrOff;
+            const int ksteps = min(LRC, p.rank - c * LRC) / 16;
+            for (int ks = 0; ks < ksteps; ++ks) {
+              const uint32_t a_addr = lr + (uint32_t)((ks >> 2) * (C::kLrT / 2) + (ks & 3) * 32);
+              const uint32_t b_addr = lr + (uint32_t)(C::kLrT + ks * 2048);
+              mma_bf16_ss_pair(tmem + C::kLrCol, smem_desc_kmajor_sw128(a_addr),
+                               smem_desc_mnmajor_sw128(b_addr, 8192, 1024), idesc_lr, (c | ks) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair_mc(&bar->lr_empty, 0x3);
+          }
         }
         tc_commit_pair_mc(&bar->acc_full, 0x3);
       }
@@ -288,9 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 16) {
     // ------------------------------------------------ widen (INT4) + epilogue
-    // warps 0-7 widen A (TMEM) and run the epilogue; warps 8-15 widen B (smem).
-    // Two sets of warps take alternate k-blocks (set 0 even, set 1 odd) so
-    // that each warp has two MMA k-blocks of time per widen.
+    // warps 0-7 widen A (TMEM), warps 8-15 widen B (smem); two sets of warps
+    // take alternate k-blocks (set 0 even, set 1 odd) so that each warp has
+    // two MMA k-blocks of time per widen.  All 16 run the epilogue.
     const bool is_a = warp < 8;
     const int set = (warp >> 2) & 1;
     const int quad = warp & 3;
@@ -304,7 +380,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         set_device_error(prm.err, kDevErrTimeoutFull);
         return false;
       }
-      const uint32_t src = sbase + (uint32_t)(ps * kPkStage + (is_a ? 0 : kPkA) + r * (BK / 2));
+      if (!is_a && r >= BNH) {
+        // B has only BNH rows per CTA: surplus lanes only take part in the
+        // warp-level hand-offs
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->tma_empty[ps]);
+        if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
+          set_device_error(prm.err, kDevErrTimeoutEmpty);
+          return false;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
+        return true;
+      }
+      const uint32_t src = sbase + (uint32_t)(ps * C::kPkStage + (is_a ? 0 : C::kPkA) + r * (BK / 2));
       const uint32_t rsw64 = (uint32_t)((r >> 1) & 3);
       uint4 pk[4];
 #pragma unroll
@@ -330,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
       } else {
         const uint32_t row =
-            sbase + (uint32_t)(kPkRingBytes + u * kWideB + (r >> 3) * 1024 + (r & 7) * 128);
+            sbase + (uint32_t)(PS * C::kPkStage + u * C::kWideB + (r >> 3) * 1024 + (r & 7) * 128);
         const uint32_t rsw128 = (uint32_t)(r & 7);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -346,13 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    // epilogue of tile i: each of the 16 warps drains 64 accumulator columns
-    // of its TMEM lane quadrant into registers, releases the accumulator to
-    // the next tile's MMAs, then dequantizes, adds the low-rank term and the
-    // bias and writes bf16 through TMA stores.
-    const int cq = warp >> 2;                         // column quarter (64 columns)
-    const uint32_t stage_out = sbase + (uint32_t)(ring_bytes<PACKED>() + warp * kStageTile);
-    float* vec_base = reinterpret_cast<float*>(smem_raw + (sbase - raw) + ring_bytes<PACKED>() + kOutStageBytes);
+    // epilogue of tile i: each of the 16 warps drains its TMEM lane quadrant's
+    // share of the accumulator columns (and of the low-rank accumulator) into
+    // registers, releases the accumulators to the next tile's MMAs, then
+    // dequantizes, adds the low-rank term and the bias and writes bf16
+    // through TMA stores.
+    const int cq = warp >> 2;                         // column quarter
+    const uint32_t stage_out = sbase + (uint32_t)(C::kOutOff + warp * kStageTile);
+    float* vec_base = reinterpret_cast<float*>(smem_raw + (sbase - raw) + C::kVecOff);
     const uint32_t sw64 = (uint32_t)((lane >> 1) & 3);
     auto epilogue = [&](int i) {
       const int m_row0 = tile_m(i) + quad * 32;
@@ -372,16 +462,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bar->acc_full, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
       tc_fence_after();
       uint32_t v[2][32];
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + kAccCol + (uint32_t)(cq * 64);
-      tmem_ld_32x32b_x32(taddr, v[0]);
-      tmem_ld_32x32b_x32(taddr + 32, v[1]);
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(cq * C::kColsPerWarp);
+      tmem_ld_32x32b_x32(taddr + kAccCol, v[0]);
+      if (LR)
+        tmem_ld_32x32b_x32(taddr + C::kLrCol, v[1]);
+      else
+        tmem_ld_32x32b_x32(taddr + kAccCol + 32, v[1]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(&bar->acc_empty, 0);
+      constexpr int kChunks = LR ? 1 : 2;
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int c0 = cq * 64 + ch * 32;
+      for (int ch = 0; ch < kChunks; ++ch) {
+        const int c0 = cq * C::kColsPerWarp + ch * 32;
         const int n = n_pair + c0;
         if (n >= p.N) continue;  // warp-uniform
         const int nv = min(32, p.N - n);
@@ -394,31 +488,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               dd[c] = make_uint4((uint32_t)((int)vv[4 * c] >> kShift), (uint32_t)((int)vv[4 * c + 1] >> kShift),
                                  (uint32_t)((int)vv[4 * c + 2] >> kShift), (uint32_t)((int)vv[4 * c + 3] >> kShift));
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int acc = static_cast<int>(vv[j]) >> kShift;
-          vv[j] = __float_as_uint(
-              __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), sa), s_sw[c0 + j]), p.inv_group));
-        }
-        if (p.rank > 0 && mok) {
-          const uint16_t* trow = p.T + m * p.rank;
-#pragma unroll 1
-          for (int jj = 0; jj < p.rank; ++jj) {
-            const float t = bf16_bits_to_float(trow[jj]);
-            const uint16_t* l2 = p.L2 + (long)jj * p.N + n;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nv)
-                vv[j] = __float_as_uint(__fmaf_rn(t, bf16_bits_to_float(__ldg(l2 + j)), __uint_as_float(vv[j])));
-          }
-        }
         uint32_t o[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float y0 = __fadd_rn(__uint_as_float(vv[2 * j]), s_bias[c0 + 2 * j]);
-          const float y1 = __fadd_rn(__uint_as_float(vv[2 * j + 1]), s_bias[c0 + 2 * j + 1]);
-          __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-          o[j] = *reinterpret_cast<uint32_t*>(&h);
+          float y[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int jj = 2 * j + h;
+            float t = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(vv[jj]) >> kShift), sa),
+                                          s_sw[c0 + jj]),
+                                p.inv_group);
+            if (LR) t = __fadd_rn(t, __uint_as_float(v[1][jj]));
+            y[h] = __fadd_rn(t, s_bias[c0 + jj]);
+          }
+          __nv_bfloat162 hb = __floats2bfloat162_rn(y[0], y[1]);
+          o[j] = *reinterpret_cast<uint32_t*>(&hb);
         }
         // stage the warp's 32 x 32 tile and let TMA write it (rows past M and
         // columns past N are dropped by the tensor map bounds)
@@ -480,56 +564,54 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major uint8 matrix [rows, cols] as a 2-D tensor map with a
-// (box_cols x box_rows) box; rows past the end read as zero.
-bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                  uint32_t box_rows, CUtensorMapSwizzle swz) {
+// Row-major matrix [rows, cols] of 1- or 2-byte elements as a 2-D tensor map
+// with a (box_cols x box_rows) box; elements past the ends read as zero.
+bool make_tmap(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* base, uint64_t rows,
+               uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major bf16 matrix [rows, cols] as a 2-D tensor map (box_cols x box_rows).
-bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                    uint32_t box_rows, CUtensorMapSwizzle swz) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <bool PACKED>
+template <bool PACKED, bool LR>
 cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
+  using C = Cfg<PACKED, LR>;
+  auto kern = gemm_kernel<PACKED, LR>;
   static int configured[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !configured[dev]) {
-    e = cudaFuncSetAttribute(gemm_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<PACKED>());
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  CUtensorMap tA, tB;
+  CUtensorMap tA, tB, tY, tT, tL2;
   const uint64_t row_bytes = PACKED ? (uint64_t)a.K / 2 : (uint64_t)a.K;
   const uint32_t box_cols = PACKED ? BK / 2 : BK;
   const CUtensorMapSwizzle swz = PACKED ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  CUtensorMap tY;
-  if (!make_tmap_u8(&tA, a.A, (uint64_t)a.M, row_bytes, box_cols, BM, swz) ||
-      !make_tmap_u8(&tB, a.B, (uint64_t)a.N, row_bytes, box_cols, BNH, swz) ||
-      !make_tmap_bf16(&tY, a.Y, (uint64_t)a.M, (uint64_t)a.N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+  if (!make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.A, (uint64_t)a.M, row_bytes, box_cols, BM, swz) ||
+      !make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.B, (uint64_t)a.N, row_bytes, box_cols, C::BNH, swz) ||
+      !make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.Y, (uint64_t)a.M, (uint64_t)a.N, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  const int pairs = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+  if (LR) {
+    // T [M, r]: 64-rank x 128-row boxes; L2 [r, N]: BNH-column x 128-rank boxes
+    if (!make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T, (uint64_t)a.M, (uint64_t)a.rank, 64, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&tL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.L2, (uint64_t)a.rank, (uint64_t)a.N, C::BNH, LRC,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
+    tT = tY;
+    tL2 = tY;
+  }
+  const int pairs = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + C::BN - 1) / C::BN);
   static int sm_count[64] = {0};
   if (dev < 64 && !sm_count[dev]) {
     int n = 0;
@@ -540,7 +622,7 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * std::min(pairs, sms / 2), 1, 1);   // persistent: one pair per TPC
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes<PACKED>();
+  cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -552,7 +634,7 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   Params prm{a, err};
-  e = cudaLaunchKernelEx(&cfg, gemm_kernel<PACKED>, prm, tA, tB, tY);
+  e = cudaLaunchKernelEx(&cfg, kern, prm, tA, tB, tY, tT, tL2);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -564,7 +646,8 @@ unsigned int* device_error_word();
 cudaError_t launch_gemm(const GemmArgs& a, bool packed_int4, cudaStream_t st) {
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorInvalidDevicePointer;
-  return packed_int4 ? launch_impl<true>(a, err, st) : launch_impl<false>(a, err, st);
+  if (!packed_int4) return launch_impl<false, false>(a, err, st);
+  return a.rank > 0 ? launch_impl<true, true>(a, err, st) : launch_impl<true, false>(a, err, st);
 }
 
 }  // namespace w4a4
