@@ -544,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
+  __syncwarp();   // single-lane roles rejoin their warps before the aligned cluster barrier
   cluster_sync();
   if (warp == kTmaWarp) {
     tc_fence_after();

@@ -1,14 +1,22 @@
-// Low-rank down-projection T = X L1 of the SVDQuant branch.
+// Low-rank down-projection T = X L1 of the SVDQuant branch (A4).
 //
 // Method: "Krea 2 Turbo - SVDQuant" (sweettea.co), "What's included" -- a
 // low-rank correction branch runs in parallel with the 4-bit matmul; reading:
 // the branch takes the unrotated bf16 activations, T = X L1 accumulates in
-// fp32 and is stored as bf16 for the up-projection folded into the GEMM
-// epilogue.
+// fp32 and is stored as bf16 for the up-projection folded into the GEMM.
 //
-// Shared-memory tiled fp32 kernel: a CTA computes a 64 x 64 tile of T with
-// 256 threads (4 x 4 outputs each), staging 64 x 32 slabs of X and 32 x 64
-// slabs of L1.  Rank r <= 256 keeps this a thin product (2 M K r flops).
+// A thin product (N = rank <= 256), so the kernel splits K over a cluster of
+// S CTAs (S <= 8) to put enough SMs on the activations: each CTA streams a
+// 128-row tile of X (K-major, 128-byte swizzle) and the matching rows of L1
+// (N-major, 128-byte swizzle) through a 4-deep TMA ring and accumulates its K
+// slice with tcgen05.mma kind::f16 into TMEM.  The fp32 partials are drained
+// into each CTA's shared memory and reduced through distributed shared memory
+// in a fixed CTA order (deterministic, no global scratch); each CTA writes
+// 128/S rows of T.
+#include <algorithm>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -18,66 +26,254 @@ namespace w4a4 {
 
 namespace {
 
-constexpr int TM = 64, TN = 64, TK = 32;
+constexpr int BM = 128;        // rows of X per tile
+constexpr int BKL = 64;        // K per stage (128 bytes of bf16: one swizzle row)
+constexpr int NST = 4;         // TMA stages
+constexpr int kThreads = 128;
 
-__device__ __forceinline__ float bf(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+struct LrBarriers {
+  uint64_t full[NST];
+  uint64_t empty[NST];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+};
 
-__global__ void __launch_bounds__(256) lowrank_down_kernel(const uint16_t* __restrict__ X,
-                                                           const uint16_t* __restrict__ L1, int M, int K, int r,
-                                                           uint16_t* __restrict__ T) {
-  __shared__ float xs[TK][TM + 1];
-  __shared__ float ls[TK][TN + 1];
-  grid_launch_dependents();
-  const int m0 = blockIdx.y * TM, j0 = blockIdx.x * TN;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += TK) {
-    for (int i = threadIdx.x; i < TM * TK; i += 256) {
-      const int mm = i / TK, kk = i % TK;
-      const long m = m0 + mm;
-      xs[kk][mm] = (m < M) ? bf(X[m * K + k0 + kk]) : 0.0f;
-    }
-    for (int i = threadIdx.x; i < TK * TN; i += 256) {
-      const int kk = i / TN, jj = i % TN;
-      const int j = j0 + jj;
-      ls[kk][jj] = (j < r) ? bf(L1[(long)(k0 + kk) * r + j]) : 0.0f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < TK; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) b[i] = ls[kk][tx * 4 + i];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int jv = 0; jv < 4; ++jv) acc[i][jv] = __fmaf_rn(a[i], b[jv], acc[i][jv]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long m = m0 + ty * 4 + i;
-    if (m >= M) continue;
-#pragma unroll
-    for (int jv = 0; jv < 4; ++jv) {
-      const int j = j0 + tx * 4 + jv;
-      if (j < r) {
-        __nv_bfloat16 h = __float2bfloat16_rn(acc[i][jv]);
-        T[m * r + j] = *reinterpret_cast<uint16_t*>(&h);
+struct LrParams {
+  uint16_t* T;
+  int M, K, r, S;
+  unsigned int* err;
+};
+
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    lowrank_down_kernel(const LrParams p, const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmL1) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  const int rb = (p.r + 63) / 64;                       // 64-rank blocks of L1
+  const int kAB = BM * BKL * 2;                         // X stage: 16 KB
+  const int kBB = rb * BKL * 128;                       // L1 stage: rb boxes of 64 K-rows x 128 bytes
+  const int kStage = kAB + kBB;
+  const int part_pitch = p.r * 4 + 16;                  // fp32 partial row pitch (padded)
+  const int data = max(NST * kStage, BM * part_pitch);
+  LrBarriers* bar = reinterpret_cast<LrBarriers*>(smem_raw + (sbase - raw) + data);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_ctarank();
+  const int S = p.S;
+  const int m0 = (blockIdx.x / S) * BM;
+  const int nkb = p.K / BKL;
+  const int kb0 = (int)crank * nkb / S;
+  const int kb1 = ((int)crank + 1) * nkb / S;
+  uint32_t ncols = 32;
+  while ((int)ncols < p.r) ncols <<= 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmL1);
+      for (int s = 0; s < NST; ++s) {
+        mbar_init(&bar->full[s], 1);
+        mbar_init(&bar->empty[s], 1);
       }
+      mbar_init(&bar->acc_full, 1);
+      fence_mbar_init();
+    }
+  } else if (warp == 2) {
+    tmem_alloc(&bar->tmem_base, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+  // X may come from the previous kernel of the stream, and the previous
+  // layer may still read this T
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------- TMA
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&bar->empty[s], ph ^ 1u)) {
+        set_device_error(p.err, kDevErrTimeoutEmpty);
+        break;
+      }
+      const uint32_t st = sbase + (uint32_t)(s * kStage);
+      mbar_arrive_expect_tx(&bar->full[s], (uint32_t)kStage);
+      tma_load_2d(st, &tmX, kb * BKL, m0, &bar->full[s]);
+      for (int b = 0; b < rb; ++b)
+        tma_load_2d(st + kAB + b * (BKL * 128), &tmL1, b * 64, kb * BKL, &bar->full[s]);
+      if (++s == NST) { s = 0; ph ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------- MMA
+    const uint32_t idesc = idesc_bf16(BM, p.r, false, true);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&bar->full[s], ph)) {
+        set_device_error(p.err, kDevErrTimeoutFull);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = sbase + (uint32_t)(s * kStage);
+#pragma unroll
+      for (int ks = 0; ks < BKL / 16; ++ks)
+        mma_bf16_ss(tmem, smem_desc_kmajor_sw128(st + (uint32_t)(ks * 32)),
+                    smem_desc_mnmajor_sw128(st + (uint32_t)(kAB + ks * 2048), BKL * 128, 1024), idesc,
+                    (kb > kb0 || ks > 0) ? 1u : 0u);
+      tc_commit(&bar->empty[s]);
+      if (++s == NST) { s = 0; ph ^= 1u; }
+    }
+    tc_commit(&bar->acc_full);
+  }
+
+  // --------------------------------------------- drain partials to smem
+  __syncwarp();   // lanes 0 of warps 0 and 1 rejoin before the warp-wide TMEM loads
+  if (!mbar_wait(&bar->acc_full, 0)) set_device_error(p.err, kDevErrTimeoutAcc);
+  tc_fence_after();
+  const int row = warp * 32 + lane;
+  const uint32_t part = sbase + (uint32_t)(row * part_pitch);
+  for (int c0 = 0; c0 < p.r; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+    tmem_wait_ld();
+    if (kb1 == kb0) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0u;   // an empty K slice contributes zero
+    }
+    const int nv = min(32, p.r - c0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (4 * q < nv)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(part + (uint32_t)((c0 + 4 * q) * 4)),
+                     "r"(v[4 * q]), "r"(v[4 * q + 1]), "r"(v[4 * q + 2]), "r"(v[4 * q + 3])
+                     : "memory");
+  }
+  tc_fence_before();
+  cluster_sync();
+
+  // --------------------------------------------- reduce across the cluster
+  const int rows_per = BM / S;
+  const int vec_per_row = p.r / 4;
+  for (int item = threadIdx.x; item < rows_per * vec_per_row; item += kThreads) {
+    const int rr = (int)crank * rows_per + item / vec_per_row;
+    const int c = (item % vec_per_row) * 4;
+    const uint32_t local = sbase + (uint32_t)(rr * part_pitch + c * 4);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < S; ++s) {
+      const uint4 w = ld_cluster_v4(map_to_rank(local, (uint32_t)s));
+      acc[0] = __fadd_rn(acc[0], __uint_as_float(w.x));
+      acc[1] = __fadd_rn(acc[1], __uint_as_float(w.y));
+      acc[2] = __fadd_rn(acc[2], __uint_as_float(w.z));
+      acc[3] = __fadd_rn(acc[3], __uint_as_float(w.w));
+    }
+    const long m = (long)m0 + rr;
+    if (m < p.M) {
+      __nv_bfloat162 a = __floats2bfloat162_rn(acc[0], acc[1]);
+      __nv_bfloat162 b = __floats2bfloat162_rn(acc[2], acc[3]);
+      uint2 o = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+      *reinterpret_cast<uint2*>(p.T + m * p.r + c) = o;
     }
   }
+  cluster_sync();   // partials stay readable until every CTA has reduced
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_lr() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+               uint32_t box_rows) {
+  auto fn = encode_fn_lr();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
+unsigned int* device_error_word();
+
 cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
                                 cudaStream_t st) {
-  dim3 grid((r + TN - 1) / TN, (M + TM - 1) / TM);
-  lowrank_down_kernel<<<grid, 256, 0, st>>>(X, L1, M, K, r, T);
+  unsigned int* err = device_error_word();
+  if (!err) return cudaErrorInvalidDevicePointer;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int m_tiles = (M + BM - 1) / BM;
+  const int nkb = K / BKL;
+  int S = 1;
+  while (S < 8 && m_tiles * S * 2 <= sms && S * 2 <= nkb) S *= 2;   // about one CTA per SM
+  const int rb = (r + 63) / 64;
+  const int stage = BM * BKL * 2 + rb * BKL * 128;
+  const int data = std::max(NST * stage, BM * (r * 4 + 16));
+  const int smem = data + (int)sizeof(LrBarriers) + 1024;
+  static int attr_smem[64] = {0};
+  if (dev < 64 && attr_smem[dev] < smem) {
+    e = cudaFuncSetAttribute(lowrank_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e != cudaSuccess) return e;
+    attr_smem[dev] = 232448;
+  }
+  CUtensorMap tX, tL1;
+  if (!tmap_bf16(&tX, X, (uint64_t)M, (uint64_t)K, BKL, BM) ||
+      !tmap_bf16(&tL1, L1, (uint64_t)K, (uint64_t)r, 64, BKL))
+    return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(m_tiles * S, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  LrParams prm{T, M, K, r, S, err};
+  e = cudaLaunchKernelEx(&cfg, lowrank_down_kernel, prm, tX, tL1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
