@@ -34,6 +34,10 @@
 //   warp 17     (even CTA) one thread issues the pair MMAs and commits each
 //               stage to the barriers of both CTAs; (odd CTA) relays the
 //               arrival of TMA-only operands to the even CTA.
+//   warp 18     (even CTA) polls the stage barriers and releases each stage
+//               to warp 17 through a named barrier: the issuing warp never
+//               reads shared memory, which would stall it behind its own
+//               queued MMAs and leave the tensor pipe idle between stages.
 //   warps 0-15  epilogue: tcgen05.ld, dequant, low-rank, bias, bf16 TMA
 //               stores.
 // The kernel is persistent: one pair per TPC walks its output tiles, and the
@@ -60,9 +64,11 @@ namespace {
 
 constexpr int BM = 128;          // A rows per CTA; the pair covers 256
 constexpr int BK = 128;          // codes per k-block
-constexpr int kThreads = 576;    // 18 warps
+constexpr int kThreads = 608;    // 19 warps
 constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
+constexpr int kWaitWarp = 18;
+constexpr int kIssueBar = 2;     // named barrier: MMA warp + waiter warp
 constexpr int PS = 5;            // packed TMA stages
 constexpr int US = 6;            // widened stages
 constexpr int S8 = 5;            // INT8 TMA stages
@@ -148,6 +154,20 @@ __device__ __forceinline__ void widen16(const uint4 p, uint4& c0, uint4& c1) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// int32 accumulator -> float.  Widened products carry a factor 2^8; after the
+// shift |t| <= 64 K <= 2^21, so t is recovered exactly from the mantissa of
+// 1.5 * 2^23 + t (two full-rate ALU operations instead of a conversion-unit
+// I2F).  The INT8 accumulator can exceed 2^22 and is rounded by I2F.
+template <bool PACKED>
+__device__ __forceinline__ float acc_to_float(uint32_t v) {
+  if constexpr (PACKED) {
+    const int t = static_cast<int>(v) >> 8;
+    return __fsub_rn(__int_as_float(t + 0x4B400000), 12582912.0f);
+  } else {
+    return __int2float_rn(static_cast<int>(v));
+  }
+}
 
 template <bool PACKED, bool LR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -286,81 +306,117 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (leader && lane == 0) {
+    if (leader) {
       // ---------------------------------------------------------------- MMA
+      // The whole warp walks the stages; lane 0 issues.  This warp never
+      // polls an mbarrier: a shared-memory read here would queue behind the
+      // MMAs already issued and leave the tensor pipe idle between stages.
+      // The waiter warp polls the barriers and releases each stage through
+      // a named barrier (bar.red also carries its timeout flag).
       constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
       constexpr uint32_t idesc_lr = idesc_bf16(2 * BM, BN, false, true);
       constexpr int NS = PACKED ? US : S8;
-      int s = 0, lr_n = 0;
-      uint32_t ph = 0;
+      int s = 0;
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
-        // the accumulators are free once both CTAs' epilogues have read tile i-1
-        if (i > 0 && !mbar_wait(&bar->acc_empty, (uint32_t)(i - 1) & 1u)) {
-          set_device_error(prm.err, kDevErrTimeoutAcc);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
-          if (PACKED) {
-            if (!mbar_wait(&bar->full[s], ph)) {
-              set_device_error(prm.err, kDevErrTimeoutFull);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
-#pragma unroll
-            for (int ks = 0; ks < BK / 32; ++ks)
-              mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8),
-                             smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
-                             (kb | ks) != 0 ? 1u : 0u);
-            tc_commit_pair_mc(&bar->empty[s], 0x3);
-          } else {
-            if (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait(&bar->full[s], ph)) {
-              set_device_error(prm.err, kDevErrTimeoutFull);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a_stage = sbase + (uint32_t)(s * C::kI8Stage);
-#pragma unroll
-            for (int ks = 0; ks < BK / 32; ++ks)
-              mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
-                             smem_desc_kmajor_sw128(a_stage + C::kI8A + (uint32_t)(ks * 32)), idesc,
-                             (kb | ks) != 0 ? 1u : 0u);
-            tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
+          if (named_barrier_or(kIssueBar, 64, false)) {
+            ok = false;
+            break;
           }
-          if (++s == NS) { s = 0; ph ^= 1u; }
+          tc_fence_after();
+          if (lane == 0) {
+            if (PACKED) {
+              const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
+#pragma unroll
+              for (int ks = 0; ks < BK / 32; ++ks)
+                mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8),
+                               smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+              tc_commit_pair_mc(&bar->empty[s], 0x3);
+            } else {
+              const uint32_t a_stage = sbase + (uint32_t)(s * C::kI8Stage);
+#pragma unroll
+              for (int ks = 0; ks < BK / 32; ++ks)
+                mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
+                               smem_desc_kmajor_sw128(a_stage + C::kI8A + (uint32_t)(ks * 32)), idesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+              tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
+            }
+          }
+          __syncwarp();
+          if (++s == NS) s = 0;
         }
         if (LR) {
           // T L2 into the fp32 accumulator: A = T (K-major, 128-byte
           // swizzle, k-step 16 ranks = 32 bytes), B = L2 (N-major, 128-byte
           // swizzle, k-step 16 ranks = two 8-row atoms)
-          for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
-            if (!mbar_wait(&bar->lr_full, (uint32_t)lr_n & 1u) || !mbar_wait(&bar->lr_ready, (uint32_t)lr_n & 1u)) {
-              set_device_error(prm.err, kDevErrTimeoutFull);
+          for (int c = 0; c < lr_chunks && ok; ++c) {
+            if (named_barrier_or(kIssueBar, 64, false)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t lr = sbase + (uint32_t)C::kLrOff;
-            const int ksteps = min(LRC, p.rank - c * LRC) / 16;
-            for (int ks = 0; ks < ksteps; ++ks) {
-              const uint32_t a_addr = lr + (uint32_t)((ks >> 2) * (C::kLrT / 2) + (ks & 3) * 32);
-              const uint32_t b_addr = lr + (uint32_t)(C::kLrT + ks * 2048);
-              mma_bf16_ss_pair(tmem + C::kLrCol, smem_desc_kmajor_sw128(a_addr),
-                               smem_desc_mnmajor_sw128(b_addr, 8192, 1024), idesc_lr, (c | ks) != 0 ? 1u : 0u);
+            if (lane == 0) {
+              const uint32_t lr = sbase + (uint32_t)C::kLrOff;
+              const int ksteps = min(LRC, p.rank - c * LRC) / 16;
+              for (int ks = 0; ks < ksteps; ++ks) {
+                const uint32_t a_addr = lr + (uint32_t)((ks >> 2) * (C::kLrT / 2) + (ks & 3) * 32);
+                const uint32_t b_addr = lr + (uint32_t)(C::kLrT + ks * 2048);
+                mma_bf16_ss_pair(tmem + C::kLrCol, smem_desc_kmajor_sw128(a_addr),
+                                 smem_desc_mnmajor_sw128(b_addr, 8192, 1024), idesc_lr, (c | ks) != 0 ? 1u : 0u);
+              }
+              tc_commit_pair_mc(&bar->lr_empty, 0x3);
             }
-            tc_commit_pair_mc(&bar->lr_empty, 0x3);
+            __syncwarp();
           }
         }
-        tc_commit_pair_mc(&bar->acc_full, 0x3);
+        if (ok && lane == 0) tc_commit_pair_mc(&bar->acc_full, 0x3);
+        __syncwarp();
       }
       // drain: every MMA issued so far has completed before teardown
-      tc_commit_pair_mc(&bar->drain, 0x1);
-      if (!mbar_wait(&bar->drain, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
+      if (lane == 0) {
+        tc_commit_pair_mc(&bar->drain, 0x1);
+        if (!mbar_wait(&bar->drain, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
+      }
+      __syncwarp();
+    }
+  } else if (warp == kWaitWarp) {
+    if (leader) {
+      // ------------------------------------------------------------- waiter
+      // Polls, in the issuer's order, every barrier an MMA stage depends on
+      // and releases the stage to the issuer warp through the named barrier.
+      constexpr int NS = PACKED ? US : S8;
+      int s = 0, lr_n = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        for (int kb = 0; kb < nk; ++kb) {
+          // the accumulators are free once both CTAs' epilogues have read tile i-1
+          bool late = kb == 0 && i > 0 && !mbar_wait(&bar->acc_empty, (uint32_t)(i - 1) & 1u);
+          if (late) {
+            if (lane == 0) set_device_error(prm.err, kDevErrTimeoutAcc);
+          } else if (PACKED ? !mbar_wait(&bar->full[s], ph)
+                            : (!mbar_wait(&bar->tma_full[s], ph) || !mbar_wait(&bar->full[s], ph))) {
+            late = true;
+            if (lane == 0) set_device_error(prm.err, kDevErrTimeoutFull);
+          }
+          if (named_barrier_or(kIssueBar, 64, late)) {
+            ok = false;
+            break;
+          }
+          if (++s == NS) { s = 0; ph ^= 1u; }
+        }
+        for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
+          const bool late = !mbar_wait(&bar->lr_full, (uint32_t)lr_n & 1u) ||
+                            !mbar_wait(&bar->lr_ready, (uint32_t)lr_n & 1u);
+          if (late && lane == 0) set_device_error(prm.err, kDevErrTimeoutFull);
+          if (named_barrier_or(kIssueBar, 64, late)) {
+            ok = false;
+            break;
+          }
+        }
+      }
     }
   } else if (warp < 16) {
     // ------------------------------------------------ widen (INT4) + epilogue
@@ -398,8 +454,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4 pk[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw64) << 4));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->tma_empty[ps]);
+      // Hand the packed stage back to TMA only once every lane's loads have
+      // returned: the arrive is made data-dependent on all loaded words (an
+      // mbarrier arrive by itself does not wait for this warp's outstanding
+      // shared-memory loads, and the next bulk copy into the stage would
+      // overwrite data not yet read).  Exactly one lane arrives whatever the
+      // value.
+      uint32_t seen = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) seen ^= pk[c].x ^ pk[c].y ^ pk[c].z ^ pk[c].w;
+      seen = __reduce_or_sync(0xffffffffu, seen);
+      if (lane == (seen == 0x9E3779B9u ? 1 : 0)) mbar_arrive(&bar->tma_empty[ps]);
       if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
         set_device_error(prm.err, kDevErrTimeoutEmpty);
         return false;
@@ -452,7 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (threadIdx.x < BN) {
         const int j = threadIdx.x;
         const int n = n_pair + j;
-        s_sw[j] = n < p.N ? __ldg(p.b_scale + n) : 0.0f;
+        // 1/g is a power of two: folding it into the column scale is exact
+        // (s_w / g stays a normal float for any scale above 2^-119)
+        s_sw[j] = n < p.N ? __ldg(p.b_scale + n) * p.inv_group : 0.0f;
         s_bias[j] = (p.bias && n < p.N) ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f;
       }
       named_barrier_sync(1, 512);
@@ -490,19 +557,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint32_t o[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float y[2];
+        for (int q = 0; q < 8; ++q) {
+          const float4 w4 = *reinterpret_cast<const float4*>(s_sw + c0 + 4 * q);
+          const float4 b4 = *reinterpret_cast<const float4*>(s_bias + c0 + 4 * q);
+          const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+          float y[4];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int jj = 2 * j + h;
-            float t = __fmul_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(vv[jj]) >> kShift), sa),
-                                          s_sw[c0 + jj]),
-                                p.inv_group);
+          for (int h = 0; h < 4; ++h) {
+            const int jj = 4 * q + h;
+            float t = __fmul_rn(__fmul_rn(acc_to_float<PACKED>(vv[jj]), sa), wv[h]);
             if (LR) t = __fadd_rn(t, __uint_as_float(v[1][jj]));
-            y[h] = __fadd_rn(t, s_bias[c0 + jj]);
+            y[h] = __fadd_rn(t, bv[h]);
           }
-          __nv_bfloat162 hb = __floats2bfloat162_rn(y[0], y[1]);
-          o[j] = *reinterpret_cast<uint32_t*>(&hb);
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
+          o[2 * q] = *reinterpret_cast<uint32_t*>(&h0);
+          o[2 * q + 1] = *reinterpret_cast<uint32_t*>(&h1);
         }
         // stage the warp's 32 x 32 tile and let TMA write it (rows past M and
         // columns past N are dropped by the tensor map bounds)
