@@ -267,52 +267,86 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
   cp_async_wait<0>();
 }
 
+// Launch shape: rows per block R (R * K/g threads, at most MAXT) and the
+// number of resident CTAs decide how many waves the persistent grid walks.
+// Every R is tried and the one with the least modelled time kept: a wave
+// costs the larger of a fixed memory latency and its bytes at HBM rate, and
+// the last wave costs as much as a full one.  (M = 4608, K = 3072, g = 128:
+// R = 5 gives 922 blocks on 444 CTAs -- three waves, the last 8% full;
+// R = 4 gives 1152 blocks on 592 CTAs -- two waves.)
+struct RqShape {
+  int rows_per_blk, threads, smem, grid;
+};
+
+template <int G, bool ROT, int QMAX, int MAXT>
+cudaError_t pick_shape(int M, int K, int dev, RqShape& out) {
+  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT>;
+  const int gpr = K / G;
+  const int max_r = gpr >= MAXT ? 1 : MAXT / gpr;
+  int sms = 148;
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  double best = 1e30;
+  for (int r = max_r; r >= 1; --r) {
+    const int threads = ((r * gpr + 31) / 32) * 32;
+    if (threads > MAXT) continue;
+    const int smem = kStages * r * gpr * group_stride<G>();
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess) return e;
+    per_sm = per_sm < 1 ? 1 : per_sm;
+    const long nblk = (M + r - 1) / r;
+    const long resident = (long)sms * per_sm;
+    const long grid = nblk < resident ? nblk : resident;
+    const long waves = (nblk + grid - 1) / grid;
+    const double wave_bytes = (double)grid * r * K * 2.0;
+    const double cost = (double)waves * (wave_bytes / 6.5e12 > 1.2e-6 ? wave_bytes / 6.5e12 : 1.2e-6);
+    if (cost < best * 0.999) {
+      best = cost;
+      out = RqShape{r, threads, smem, (int)grid};
+    }
+  }
+  return cudaSuccess;
+}
+
 template <int G, bool ROT, int QMAX, int MAXT>
 cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* scale, cudaStream_t st) {
-  const int gpr = K / G;
-  const int rows_per_blk = gpr >= MAXT ? 1 : MAXT / gpr;
-  const int threads = ((rows_per_blk * gpr + 31) / 32) * 32;
-  if (threads > MAXT) return cudaErrorInvalidConfiguration;
-  const int smem = kStages * rows_per_blk * gpr * group_stride<G>();
   auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT>;
-  static int attr_set[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int sms = 148, per_sm = 1;
-  if (dev < 64 && attr_set[dev] != smem) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem > 48 * 1024 ? smem : 48 * 1024);
+  static int attr_set[64] = {0};
+  if (dev < 64 && !attr_set[dev]) {
+    // the largest ring any shape uses (MAXT threads' groups, kStages deep)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStages * MAXT * group_stride<G>());
     if (e != cudaSuccess) return e;
-    attr_set[dev] = smem;
+    attr_set[dev] = 1;
   }
-  // occupancy of the last K seen on each device (deterministic, so a racing
-  // refresh only repeats the query)
-  static int cache_k[64] = {0}, cache_sms[64] = {0}, cache_per_sm[64] = {0};
-  if (dev < 64 && cache_k[dev] == K) {
-    sms = cache_sms[dev];
-    per_sm = cache_per_sm[dev];
+  // shape of the last (M, K) seen on each device (deterministic, so a racing
+  // refresh only repeats the search)
+  static int cache_m[64] = {0}, cache_k[64] = {0};
+  static RqShape cache_shape[64];
+  RqShape sh;
+  if (dev < 64 && cache_m[dev] == M && cache_k[dev] == K) {
+    sh = cache_shape[dev];
   } else {
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess) return e;
+    if ((e = pick_shape<G, ROT, QMAX, MAXT>(M, K, dev, sh)) != cudaSuccess) return e;
     if (dev < 64) {
-      cache_sms[dev] = sms;
-      cache_per_sm[dev] = per_sm;
+      cache_shape[dev] = sh;
+      cache_m[dev] = M;
       cache_k[dev] = K;
     }
   }
-  const int nblk = (M + rows_per_blk - 1) / rows_per_blk;
-  const int grid = min(nblk, sms * max(per_sm, 1));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(threads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(sh.grid, 1, 1);
+  cfg.blockDim = dim3(sh.threads, 1, 1);
+  cfg.dynamicSmemBytes = sh.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, rows_per_blk, out, scale);
+  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, sh.rows_per_blk, out, scale);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
