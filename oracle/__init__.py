@@ -1,4 +1,4 @@
-"""CPU oracle for the W4A4 ConvRot linear layer (and the W8A8 twin).
+"""CPU oracle for the W4A4 ConvRot linear layer (and the W8A8 and W4A8 twins).
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
@@ -49,6 +49,7 @@ def _load():
         lib.oracle_rotate.argtypes = [P, L, I, I, P]
         lib.oracle_rotate.restype = I
         lib.oracle_quantize.argtypes = [P, L, I, I, P, P]
+        lib.oracle_quantize_asym4.argtypes = [P, L, I, P, P, P]
         lib.oracle_pack_int4.argtypes = [P, L, I, P]
         lib.oracle_unpack_int4.argtypes = [P, L, I, P]
         lib.oracle_int_gemm.argtypes = [P, P, L, L, I, P]
@@ -107,8 +108,22 @@ def quantize(Y: np.ndarray, qmax: int) -> tuple[np.ndarray, np.ndarray]:
     return q, s
 
 
+def quantize_asym4(Y: np.ndarray) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Per-row asymmetric 4-bit quantization with a zero point in IEEE fp32
+    -> (uint8 codes 0..15, fp32 scales, uint8 zero points)."""
+    Y = np.ascontiguousarray(Y, dtype=np.float32)
+    rows, K = Y.shape
+    q = np.empty((rows, K), dtype=np.uint8)
+    s = np.empty((rows,), dtype=np.float32)
+    z = np.empty((rows,), dtype=np.uint8)
+    _load().oracle_quantize_asym4(_ptr(Y), rows, K, _ptr(q), _ptr(s), _ptr(z))
+    return q, s, z
+
+
 def pack_int4(q: np.ndarray) -> np.ndarray:
-    q = np.ascontiguousarray(q, dtype=np.int8)
+    """Two codes per byte, even k in the low nibble (4-bit two's complement for
+    signed codes; the same bits for unsigned codes 0..15)."""
+    q = np.ascontiguousarray(q).astype(np.int8)
     rows, K = q.shape
     out = np.empty((rows, K // 2), dtype=np.uint8)
     _load().oracle_pack_int4(_ptr(q), rows, K, _ptr(out))
@@ -214,6 +229,23 @@ def linear_w4a4(X, W, g, L1=None, L2=None, bias=None):
     Y = epilogue(acc, xs, ws, g, T, L2 if T is not None else None, bias)
     return dict(x_packed=xp, x_scale=xs, x_q=xq, w_packed=wp, w_scale=ws, w_q=wq,
                 acc=acc, T=T, Y=Y)
+
+
+def quantize_w4a8_weights(W: np.ndarray, g: int):
+    """Rotate + per-output-channel asymmetric 4-bit quantize + pack (W4A8)."""
+    q, s, z = quantize_asym4(rotate(W, g))
+    return pack_int4(q), s, z, q
+
+
+def linear_w4a8(X, W, g, bias=None):
+    """W4A8 layer: rotated per-token INT8 activations (as in W8A8) times
+    rotated asymmetric 4-bit weights; acc = sum_k qa * (qw - z) exactly."""
+    xq, xs = quantize_w8(X, g)
+    wp, ws, wz, wq = quantize_w4a8_weights(W, g)
+    centered = (wq.astype(np.int16) - wz.astype(np.int16)[:, None]).astype(np.int8)
+    acc = int_gemm(xq, centered)
+    Y = epilogue(acc, xs, ws, g, None, None, bias)
+    return dict(x_q=xq, x_scale=xs, w_packed=wp, w_scale=ws, w_zero=wz, w_q=wq, acc=acc, Y=Y)
 
 
 def linear_w8a8(X, W, g, bias=None):

@@ -1,5 +1,6 @@
 /*
- * Plain CPU oracle for the W4A4 ConvRot linear layer and its W8A8 twin.
+ * Plain CPU oracle for the W4A4 ConvRot linear layer and its W8A8 and W4A8
+ * twins.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
  * call this file: only the tests, the smoke check and the benchmark's CPU
@@ -179,6 +180,47 @@ void oracle_quantize(const float *Y, long rows, int K, int qmax, int8_t *q, floa
                 if (v > qmax) v = qmax;
             }
             q[r * K + k] = (int8_t)v;
+        }
+    }
+}
+
+/* ---- asymmetric 4-bit quantization with a zero point, one pair per row ---- */
+
+/* W4A8 weights ("W4A4 and W4A8: The New Quantization Toolkit", "How the
+   toolkit tells you to choose": the W4A8 mode keeps 4-bit weights with a zero
+   point).  Per row of the rotated weights: mn = min y, mx = max y,
+   s = fl32(fl32(mx - mn) / 15), z = clamp(rint_even(fl32(-mn / s)), 0, 15),
+   q = clamp(rint_even(fl32(y / s)) + z, 0, 15) (unsigned codes; the weight
+   they stand for is (q - z) * s).  A row with mx == mn gets s = 0, z = 0 and
+   all codes 0.  Every division and rounding is a single IEEE fp32 operation. */
+void oracle_quantize_asym4(const float *Y, long rows, int K, uint8_t *q, float *scale, uint8_t *zero) {
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        const float *y = Y + r * K;
+        float mn = y[0], mx = y[0];
+        for (int k = 1; k < K; ++k) {
+            if (y[k] < mn) mn = y[k];
+            if (y[k] > mx) mx = y[k];
+        }
+        const float range = mx - mn;
+        const float s = range / 15.0f;
+        int z = 0;
+        if (s != 0.0f) {
+            const float t = (-mn) / s;
+            z = (int)nearbyintf(t);
+            if (z < 0) z = 0;
+            if (z > 15) z = 15;
+        }
+        scale[r] = s;
+        zero[r] = (uint8_t)z;
+        for (int k = 0; k < K; ++k) {
+            int v = 0;
+            if (s != 0.0f) {
+                v = (int)nearbyintf(y[k] / s) + z;
+                if (v < 0) v = 0;
+                if (v > 15) v = 15;
+            }
+            q[r * K + k] = (uint8_t)v;
         }
     }
 }

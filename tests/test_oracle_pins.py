@@ -15,6 +15,10 @@ textbook facts, library routines, closed forms and hand-derived fixtures):
     lossless (equals X W^T exactly).
   * Low-rank: W = 0 reduces the layer to (X L1) L2 + b, a NumPy fp64 product.
   * Method invariant: on outlier activations, rotation lowers the W4A4 error.
+  * W4A8 (asymmetric 4-bit weights): hand-derived binary32 fixture; minimum ->
+    code 0, maximum -> 14/15, exact zero -> zero point, monotone codes, error
+    bound; centered integer product recomputed with NumPy int64; lower error
+    than W4A4 on the same layer.
   * Planted mistakes (in copies of oracle outputs, on the CPU) are caught.
 """
 from __future__ import annotations
@@ -347,3 +351,104 @@ def test_pins_catch_planted_mistakes():
     assert q[0].tolist() == [7, 2, -2]
     away = np.sign(y / s[:, None]) * np.floor(np.abs(y / s[:, None]) + 0.5)
     assert away[0].tolist() != q[0].tolist()
+
+
+# ---------------------------------------------------------------- W4A8 (asymmetric 4-bit weights)
+def _asym_golden_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "asym_int4.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            y, sbits, z, codes = [p.strip() for p in line.split("|")]
+            rows.append((np.array([[float(v) for v in y.split()]], dtype=np.float32), int(sbits, 16), int(z),
+                         [int(v) for v in codes.split()]))
+    return rows
+
+
+def test_asym4_golden():
+    """Hand-derived binary32 cases: a half-even tie, a clamped zero point, a
+    constant row, and an exact zero."""
+    for y, sbits, z, codes in _asym_golden_rows():
+        q, s, zz = oracle.quantize_asym4(y)
+        assert int(s.view(np.uint32)[0]) == sbits
+        assert int(zz[0]) == z
+        assert q[0].tolist() == codes
+
+
+def test_asym4_extremes_zero_and_error_bound():
+    """On rows that straddle zero: the minimum maps to code 0 exactly (rint is
+    odd, so rint(min/s) + rint(-min/s) = 0), the maximum to 14 or 15, an exact
+    zero to the zero point, codes are monotone in y, and the reconstruction
+    (q - z) s is within s/2 of y (within s where a code is clamped)."""
+    rng = np.random.default_rng(31)
+    Y = (rng.standard_normal((16, 512)) * np.exp2(rng.integers(-6, 6, size=(16, 1)))).astype(np.float32)
+    Y[:, 7] = 0.0
+    q, s, z = oracle.quantize_asym4(Y)
+    for r in range(Y.shape[0]):
+        y = Y[r].astype(np.float64)
+        qi = q[r].astype(np.int64)
+        assert qi[np.argmin(y)] == 0
+        assert qi[np.argmax(y)] in (14, 15)
+        assert qi[7] == z[r]
+        order = np.argsort(y, kind="stable")
+        assert np.all(np.diff(qi[order]) >= 0)
+        err = np.abs(y - (qi - int(z[r])) * float(s[r]))
+        tol = np.where((qi == 0) | (qi == 15), 1.0, 0.5) * float(s[r]) * (1 + 2.0 ** -20)
+        assert np.all(err <= tol)
+
+
+def _unpack_unsigned(packed: np.ndarray, K: int) -> np.ndarray:
+    lo = (packed & 0xF).astype(np.int64)
+    hi = (packed >> 4).astype(np.int64)
+    out = np.empty((packed.shape[0], K), dtype=np.int64)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+@pytest.mark.parametrize("g", [0, 64, 128])
+def test_w4a8_accumulator_is_the_centered_integer_product(g):
+    """acc = sum_k qa (qw - z), recomputed with NumPy int64 from the packed
+    bytes (unpacked independently)."""
+    spec = inputs.LayerSpec("w4a8", 24, 256, 40, g if g else 128, rank=0, bias=True, seed=5, outlier_scale=50.0)
+    d = inputs.make_layer(spec)
+    out = oracle.linear_w4a8(d["X"], d["W"], g, d["bias"])
+    u = _unpack_unsigned(out["w_packed"], 256)
+    assert np.array_equal(u, out["w_q"].astype(np.int64))
+    assert u.min() >= 0 and u.max() <= 15
+    acc = out["x_q"].astype(np.int64) @ (u - out["w_zero"].astype(np.int64)[:, None]).T
+    assert np.array_equal(acc, out["acc"].astype(np.int64))
+
+
+def test_w4a8_error_below_w4a4():
+    """8-bit activations with zero-pointed 4-bit weights err less than W4A4 on
+    the same rotated layer (outliers 10x and 50-200x)."""
+    for kw in (dict(outlier_scale=10.0), {}):
+        spec = inputs.LayerSpec("q8", 128, 1024, 96, 128, rank=0, bias=False, seed=22, **kw)
+        d = inputs.make_layer(spec)
+        exact = _f32(d["X"]).astype(np.float64) @ _f32(d["W"]).astype(np.float64).T
+
+        def rel(Y):
+            return np.linalg.norm(Y - exact) / np.linalg.norm(exact)
+
+        assert rel(oracle.linear_w4a8(d["X"], d["W"], 128)["Y"]) < rel(oracle.linear_w4a4(d["X"], d["W"], 128)["Y"])
+
+
+def test_w4a8_pins_catch_planted_mistakes():
+    """A flipped zero-point sign or a zero point ignored in the product is
+    caught by the centered-product pin; rounding ties away from zero breaks
+    the golden (its 2.5 tie)."""
+    spec = inputs.LayerSpec("w4a8", 8, 256, 16, 64, rank=0, bias=False, seed=6)
+    d = inputs.make_layer(spec)
+    out = oracle.linear_w4a8(d["X"], d["W"], 64)
+    u = _unpack_unsigned(out["w_packed"], 256)
+    z = out["w_zero"].astype(np.int64)[:, None]
+    good = out["acc"].astype(np.int64)
+    assert not np.array_equal(out["x_q"].astype(np.int64) @ (u + z).T, good)
+    assert not np.array_equal(out["x_q"].astype(np.int64) @ u.T, good)
+    y, sbits, zz, codes = _asym_golden_rows()[0]
+    s = np.float32(np.uint32(sbits).view(np.float32))
+    t = (y[0] / s).astype(np.float32)
+    away = (np.sign(t) * np.floor(np.abs(t) + 0.5)).astype(np.int64) + zz
+    assert away.tolist() != codes
