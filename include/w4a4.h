@@ -178,6 +178,34 @@ w4a4_status w8a8_linear(const void* X, const int8_t* Wq, const float* w_scale, i
                         const void* bias, void* Y, void* workspace, size_t workspace_bytes,
                         w4a4_stream_t stream);
 
+/* ---------------------------------------------------------------- W4A8 twin */
+/* 4-bit weights with a zero point and 8-bit activations ("W4A4 and W4A8: The
+ * New Quantization Toolkit" (renderbob.io), "Decoding the notation" and "How
+ * the toolkit tells you to choose": the W4A8 mode keeps 4-bit weights and
+ * 8-bit activations, with a zero point on the weights).  Weights are rotated
+ * like W4A4, then quantized per output channel asymmetrically:
+ *   s = fl32(fl32(max - min) / 15), z = clamp(rint_even(fl32(-min / s)), 0, 15),
+ *   q = clamp(rint_even(fl32(y / s)) + z, 0, 15)
+ * (a row with max == min gets s = 0, z = 0 and codes 0).  Codes are stored as
+ * unsigned nibbles [N, K/2] (code 2j in the low nibble of byte j), the zero
+ * point as one byte per row.  Activations are those of the W8A8 path
+ * (w8a8_rotate_quantize_act: rotated, symmetric int8 per token).  The GEMM
+ * forms acc = sum_k xq * (wq - z) exactly in int32 and applies the W8A8
+ * epilogue ((acc * s_x) * s_w) / g + bias -> bf16.  No low-rank branch.
+ *
+ * Shapes and alignment: as w4a4_quantize_weights (weights) and w8a8_gemm
+ * (activations); w_zero needs no alignment.  w4a8_linear takes the
+ * workspace of w8a8_linear (w4a8_workspace_bytes). */
+w4a4_status w4a8_quantize_weights(const void* W, int N, int K, int group, uint8_t* Wq, float* w_scale,
+                                  uint8_t* w_zero, w4a4_stream_t stream);
+w4a4_status w4a8_gemm(const int8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale,
+                      const uint8_t* w_zero, int M, int N, int K, int group, const void* bias, void* Y,
+                      int32_t* acc_debug, w4a4_stream_t stream);
+size_t w4a8_workspace_bytes(int M, int K);
+w4a4_status w4a8_linear(const void* X, const uint8_t* Wq, const float* w_scale, const uint8_t* w_zero, int M,
+                        int N, int K, int group, const void* bias, void* Y, void* workspace,
+                        size_t workspace_bytes, w4a4_stream_t stream);
+
 /* ---------------------------------------------------------------- failures */
 /* Kernels never trap: a wait on another part of the kernel that runs past its
  * time limit (2 s) records a code in a per-device error word and lets the

@@ -36,7 +36,7 @@ def lib():
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b((?:w4a4|w8a8)_\w+)\s*\(", text, flags=re.M)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b((?:w4a4|w8a8|w4a8)_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
@@ -45,7 +45,8 @@ def test_header_declares_the_documented_entry_points():
     for n in ["w4a4_quantize_weights", "w4a4_rotate_quantize_act", "w4a4_gemm", "w4a4_linear",
               "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
               "w4a4_workspace_bytes", "w8a8_workspace_bytes", "w4a4_status_string", "w4a4_version",
-              "w4a4_get_device_error"]:
+              "w4a4_get_device_error", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear",
+              "w4a8_workspace_bytes"]:
         assert n in names
 
 
@@ -106,6 +107,27 @@ def test_gemm_validation(lib):
     bad = list(args); bad[13] = ODD                    # misaligned debug output
     assert f(*bad) == MISALIGNED
     assert lib.w8a8_gemm(A, B, C, D, 64, 4, 256, 128, NUL, E, NUL, NUL) == SHAPE
+
+
+def test_w4a8_validation(lib):
+    # quantize: the zero-point output is required
+    assert lib.w4a8_quantize_weights(A, 64, 256, 64, B, C, NUL, NUL) == INVALID
+    assert lib.w4a8_quantize_weights(A, 64, 320, 64, B, C, D, NUL) == SHAPE
+    assert lib.w4a8_quantize_weights(ODD, 64, 256, 64, B, C, D, NUL) == MISALIGNED
+    g = lib.w4a8_gemm
+    args = [A, B, C, D, E, 64, 256, 256, 128, NUL, E, NUL, NUL]
+    bad = list(args); bad[4] = NUL                     # no zero points
+    assert g(*bad) == INVALID
+    bad = list(args); bad[6] = 12                      # N not a multiple of 8
+    assert g(*bad) == SHAPE
+    bad = list(args); bad[8] = 32                      # unsupported group
+    assert g(*bad) == SHAPE
+    bad = list(args); bad[2] = ODD                     # misaligned codes
+    assert g(*bad) == MISALIGNED
+    assert lib.w4a8_workspace_bytes(5, 256) == lib.w8a8_workspace_bytes(5, 256)
+    need = lib.w4a8_workspace_bytes(16, 256)
+    assert lib.w4a8_linear(A, B, C, D, 16, 256, 256, 128, NUL, E, E, need - 1, NUL) == WORKSPACE
+    assert lib.w4a8_linear(A, B, C, NUL, 16, 256, 256, 128, NUL, E, E, need, NUL) == INVALID
 
 
 def test_linear_workspace_rules(lib):

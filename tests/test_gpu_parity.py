@@ -172,6 +172,62 @@ def test_w8a8_layer_parity(M, N, K, g):
     assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
 
 
+@pytest.mark.parametrize("N,K,g", [(264, 640, 64), (264, 640, 128), (264, 640, 0), (40, 12288, 128),
+                                   (3072, 3072, 128)])
+def test_w4a8_weight_quant_bitexact(N, K, g):
+    """Asymmetric 4-bit weights with a zero point: packed codes, scale bits
+    and zero points identical to the oracle (rows with outlier channels make
+    the minimum and maximum sit far apart)."""
+    W = inputs.random_bf16((N, K), seed=N + K + g, std=0.02)
+    W[:, 5] = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(W[:, 5]) * 60.0)
+    Wq, ws, wz = w4.w4a8_quantize_weights(dev_bf16(W), g)
+    ref_p, ref_s, ref_z, _ = oracle.quantize_w4a8_weights(W, g)
+    assert np.array_equal(ws.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+    assert np.array_equal(wz.cpu().numpy(), ref_z)
+    got = Wq.cpu().numpy()
+    assert np.array_equal(got, ref_p), f"{np.count_nonzero(got != ref_p)} code bytes differ"
+
+
+def test_w4a8_weight_quant_special_rows():
+    """A constant row (s = 0, z = 0, codes 0), an all-positive row (zero point
+    clamped to 0) and an all-negative row (clamped to 15)."""
+    K = 256
+    rows = np.stack([np.full(K, 0.5, np.float32),
+                     np.linspace(1.0, 3.0, K, dtype=np.float32),
+                     -np.linspace(1.0, 3.0, K, dtype=np.float32),
+                     np.zeros(K, np.float32)])
+    W = inputs.f32_to_bf16_bits(rows)
+    for g in (0, 64):
+        Wq, ws, wz = w4.w4a8_quantize_weights(dev_bf16(W), g)
+        ref_p, ref_s, ref_z, _ = oracle.quantize_w4a8_weights(W, g)
+        assert np.array_equal(ws.cpu().numpy().view(np.uint32), ref_s.view(np.uint32))
+        assert np.array_equal(wz.cpu().numpy(), ref_z)
+        assert np.array_equal(Wq.cpu().numpy(), ref_p)
+
+
+@pytest.mark.parametrize("M,N,K,g", [(64, 256, 256, 128), (200, 264, 384, 64), (2, 3072, 256, 128),
+                                     (257, 520, 3072, 0), (300, 768, 12288, 128)])
+def test_w4a8_layer_parity(M, N, K, g):
+    import torch
+    d = _layer(M, N, K, g, 0, True, seed=M + N + K + 2)
+    ref = oracle.linear_w4a8(d["X"], d["W"], g, d["bias"])
+    X, W, b = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    Wq, ws, wz = w4.w4a8_quantize_weights(W, g)
+    Xq, xs = w4.w8a8_rotate_quantize_act(X, g)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    Y = w4.w4a8_gemm(Xq, xs, Wq, ws, wz, g, b, acc_debug=acc)
+    torch.cuda.synchronize()
+    assert np.array_equal(Wq.cpu().numpy(), ref["w_packed"])
+    assert np.array_equal(wz.cpu().numpy(), ref["w_zero"])
+    assert np.array_equal(Xq.cpu().numpy(), ref["x_q"])
+    got = acc.cpu().numpy()
+    assert np.array_equal(got, ref["acc"]), f"{np.count_nonzero(got != ref['acc'])} accumulators differ"
+    check_output(host_f64(Y), ref["Y"], lowrank=False)
+    Y2 = w4.w4a8_linear(X, Wq, ws, wz, g, b)
+    torch.cuda.synchronize()
+    assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+
+
 def test_attn_proj_full_size_sampled():
     """The attention-projection workload at full size (M=4608, K=N=3072,
     g=128, bias), in the launch configuration the benchmark times

@@ -21,7 +21,8 @@ __all__ = [
     "w4a4_quantize_weights", "w4a4_rotate_quantize_act", "w4a4_gemm", "w4a4_linear",
     "w4a4_workspace_bytes", "w4a4_linear_noalloc", "NOALLOC_SCRATCH_BYTES",
     "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
-    "w8a8_workspace_bytes", "w4a4_get_device_error",
+    "w8a8_workspace_bytes", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear", "w4a8_workspace_bytes",
+    "w4a4_get_device_error",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -69,6 +70,10 @@ def load_library():
         "w8a8_gemm": ([P, P, P, P, I, I, I, I, P, P, P, P], S),
         "w8a8_workspace_bytes": ([I, I], Z),
         "w8a8_linear": ([P, P, P, I, I, I, I, P, P, P, Z, P], S),
+        "w4a8_quantize_weights": ([P, I, I, I, P, P, P, P], S),
+        "w4a8_gemm": ([P, P, P, P, P, I, I, I, I, P, P, P, P], S),
+        "w4a8_workspace_bytes": ([I, I], Z),
+        "w4a8_linear": ([P, P, P, P, I, I, I, I, P, P, P, Z, P], S),
         "w4a4_get_device_error": ([P, ctypes.POINTER(ctypes.c_uint)], S),
     }
     for name, (args, res) in sig.items():
@@ -228,6 +233,48 @@ def w8a8_linear(X, Wq, w_scale, group, bias=None, Y=None, workspace=None, stream
     Y = _empty((M, N), torch.bfloat16, X) if Y is None else Y
     _check("w8a8_linear", load_library().w8a8_linear(
         _ptr(X), _ptr(Wq), _ptr(w_scale), M, N, K, group, _ptr(bias), _ptr(Y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return Y
+
+
+def w4a8_quantize_weights(W, group, Wq=None, w_scale=None, w_zero=None, stream=None):
+    """Rotate + per-channel asymmetric 4-bit quantize: (packed codes [N, K/2],
+    fp32 scales [N], uint8 zero points [N])."""
+    import torch
+    N, K = W.shape
+    Wq = _empty((N, K // 2), torch.uint8, W) if Wq is None else Wq
+    w_scale = _empty((N,), torch.float32, W) if w_scale is None else w_scale
+    w_zero = _empty((N,), torch.uint8, W) if w_zero is None else w_zero
+    _check("w4a8_quantize_weights", load_library().w4a8_quantize_weights(
+        _ptr(W), N, K, group, _ptr(Wq), _ptr(w_scale), _ptr(w_zero), _stream(stream)))
+    return Wq, w_scale, w_zero
+
+
+def w4a8_gemm(Xq, x_scale, Wq, w_scale, w_zero, group, bias=None, Y=None, acc_debug=None, stream=None):
+    import torch
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    Y = _empty((M, N), torch.bfloat16, Xq) if Y is None else Y
+    _check("w4a8_gemm", load_library().w4a8_gemm(
+        _ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), _ptr(w_zero), M, N, K, group, _ptr(bias), _ptr(Y),
+        _ptr(acc_debug), _stream(stream)))
+    return Y
+
+
+def w4a8_workspace_bytes(M: int, K: int) -> int:
+    return int(load_library().w4a8_workspace_bytes(M, K))
+
+
+def w4a8_linear(X, Wq, w_scale, w_zero, group, bias=None, Y=None, workspace=None, stream=None):
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    need = w4a8_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=X.device)
+    Y = _empty((M, N), torch.bfloat16, X) if Y is None else Y
+    _check("w4a8_linear", load_library().w4a8_linear(
+        _ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(w_zero), M, N, K, group, _ptr(bias), _ptr(Y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return Y
 

@@ -98,31 +98,36 @@ const char* w4a4_status_string(w4a4_status s) {
 
 // ------------------------------------------------------------------ quantizers
 static w4a4_status quantize_rows(const void* X, int rows, int K, int group, void* out, float* scale, int qmax,
-                                 w4a4_stream_t stream) {
-  if (!X || !out || !scale) return W4A4_ERR_INVALID_ARG;
+                                 uint8_t* zero, w4a4_stream_t stream) {
+  if (!X || !out || !scale || (qmax == 15 && !zero)) return W4A4_ERR_INVALID_ARG;
   if (rows < 1) return W4A4_ERR_UNSUPPORTED_SHAPE;
   w4a4_status s = check_k_group(K, group);
   if (s != W4A4_OK) return s;
   if (!aligned16(X) || !aligned16(out) || !aligned16(scale)) return W4A4_ERR_MISALIGNED;
   if ((s = check_device()) != W4A4_OK) return s;
   return cuda_status(launch_rotate_quantize(static_cast<const uint16_t*>(X), rows, K, group, qmax,
-                                            static_cast<uint8_t*>(out), scale,
+                                            static_cast<uint8_t*>(out), scale, zero,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 w4a4_status w4a4_quantize_weights(const void* W, int N, int K, int group, uint8_t* Wq, float* w_scale,
                                   w4a4_stream_t stream) {
-  return quantize_rows(W, N, K, group, Wq, w_scale, 7, stream);
+  return quantize_rows(W, N, K, group, Wq, w_scale, 7, nullptr, stream);
 }
 
 w4a4_status w8a8_quantize_weights(const void* W, int N, int K, int group, int8_t* Wq, float* w_scale,
                                   w4a4_stream_t stream) {
-  return quantize_rows(W, N, K, group, Wq, w_scale, 127, stream);
+  return quantize_rows(W, N, K, group, Wq, w_scale, 127, nullptr, stream);
+}
+
+w4a4_status w4a8_quantize_weights(const void* W, int N, int K, int group, uint8_t* Wq, float* w_scale,
+                                  uint8_t* w_zero, w4a4_stream_t stream) {
+  return quantize_rows(W, N, K, group, Wq, w_scale, 15, w_zero, stream);
 }
 
 w4a4_status w8a8_rotate_quantize_act(const void* X, int M, int K, int group, int8_t* Xq, float* x_scale,
                                      w4a4_stream_t stream) {
-  return quantize_rows(X, M, K, group, Xq, x_scale, 127, stream);
+  return quantize_rows(X, M, K, group, Xq, x_scale, 127, nullptr, stream);
 }
 
 w4a4_status w4a4_rotate_quantize_act(const void* X, int M, int K, int group, uint8_t* Xq, float* x_scale,
@@ -139,7 +144,7 @@ w4a4_status w4a4_rotate_quantize_act(const void* X, int M, int K, int group, uin
   if (!aligned16(X) || !aligned16(Xq) || !aligned16(x_scale)) return W4A4_ERR_MISALIGNED;
   if ((s = check_device()) != W4A4_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_rotate_quantize(static_cast<const uint16_t*>(X), M, K, group, 7, Xq, x_scale, st);
+  cudaError_t e = launch_rotate_quantize(static_cast<const uint16_t*>(X), M, K, group, 7, Xq, x_scale, nullptr, st);
   if (e != cudaSuccess) return W4A4_ERR_CUDA;
   if (rank > 0) {
     e = launch_lowrank_down(static_cast<const uint16_t*>(X), static_cast<const uint16_t*>(L1), M, K, rank,
@@ -150,10 +155,12 @@ w4a4_status w4a4_rotate_quantize_act(const void* X, int M, int K, int group, uin
 }
 
 // ------------------------------------------------------------------ GEMMs
-static w4a4_status gemm_common(const void* Xq, const float* x_scale, const void* Wq, const float* w_scale, int M,
-                               int N, int K, int group, const void* T, const void* L2, int rank, const void* bias,
-                               void* Y, int32_t* acc_debug, bool packed, w4a4_stream_t stream) {
+static w4a4_status gemm_common(const void* Xq, const float* x_scale, const void* Wq, const float* w_scale,
+                               const uint8_t* w_zero, int M, int N, int K, int group, const void* T, const void* L2,
+                               int rank, const void* bias, void* Y, int32_t* acc_debug, GemmMode mode,
+                               w4a4_stream_t stream) {
   if (!Xq || !x_scale || !Wq || !w_scale || !Y) return W4A4_ERR_INVALID_ARG;
+  if (mode == GemmMode::kW4A8 && !w_zero) return W4A4_ERR_INVALID_ARG;
   w4a4_status s = check_rank(rank);
   if (s != W4A4_OK) return s;
   if (rank > 0) {
@@ -182,20 +189,29 @@ static w4a4_status gemm_common(const void* Xq, const float* x_scale, const void*
   a.bias = static_cast<const uint16_t*>(bias);
   a.Y = static_cast<uint16_t*>(Y);
   a.acc_debug = acc_debug;
-  return cuda_status(launch_gemm(a, packed, reinterpret_cast<cudaStream_t>(stream)));
+  a.w_zero = w_zero;
+  return cuda_status(launch_gemm(a, mode, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 w4a4_status w4a4_gemm(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale, int M,
                       int N, int K, int group, const void* T, const void* L2, int rank, const void* bias, void* Y,
                       int32_t* acc_debug, w4a4_stream_t stream) {
-  return gemm_common(Xq, x_scale, Wq, w_scale, M, N, K, group, T, L2, rank, bias, Y, acc_debug, true, stream);
+  return gemm_common(Xq, x_scale, Wq, w_scale, nullptr, M, N, K, group, T, L2, rank, bias, Y, acc_debug,
+                     GemmMode::kW4A4, stream);
 }
 
 w4a4_status w8a8_gemm(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale, int M,
                       int N, int K, int group, const void* bias, void* Y, int32_t* acc_debug,
                       w4a4_stream_t stream) {
-  return gemm_common(Xq, x_scale, Wq, w_scale, M, N, K, group, nullptr, nullptr, 0, bias, Y, acc_debug, false,
-                     stream);
+  return gemm_common(Xq, x_scale, Wq, w_scale, nullptr, M, N, K, group, nullptr, nullptr, 0, bias, Y, acc_debug,
+                     GemmMode::kW8A8, stream);
+}
+
+w4a4_status w4a8_gemm(const int8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale,
+                      const uint8_t* w_zero, int M, int N, int K, int group, const void* bias, void* Y,
+                      int32_t* acc_debug, w4a4_stream_t stream) {
+  return gemm_common(Xq, x_scale, Wq, w_scale, w_zero, M, N, K, group, nullptr, nullptr, 0, bias, Y, acc_debug,
+                     GemmMode::kW4A8, stream);
 }
 
 // ------------------------------------------------------------------ whole layer
@@ -208,6 +224,8 @@ size_t w8a8_workspace_bytes(int M, int K) {
   if (M < 1 || K < 1) return 0;
   return round256((size_t)M * (size_t)K) + round256((size_t)M * 4u);
 }
+
+size_t w4a8_workspace_bytes(int M, int K) { return w8a8_workspace_bytes(M, K); }
 
 w4a4_status w4a4_linear(const void* X, const uint8_t* Wq, const float* w_scale, int M, int N, int K, int group,
                         const void* L1, const void* L2, int rank, const void* bias, void* Y, void* workspace,
@@ -244,6 +262,22 @@ w4a4_status w8a8_linear(const void* X, const int8_t* Wq, const float* w_scale, i
   s = w8a8_rotate_quantize_act(X, M, K, group, Xq, xs, stream);
   if (s != W4A4_OK) return s;
   return w8a8_gemm(Xq, xs, Wq, w_scale, M, N, K, group, bias, Y, nullptr, stream);
+}
+
+w4a4_status w4a8_linear(const void* X, const uint8_t* Wq, const float* w_scale, const uint8_t* w_zero, int M,
+                        int N, int K, int group, const void* bias, void* Y, void* workspace, size_t workspace_bytes,
+                        w4a4_stream_t stream) {
+  if (!X || !Wq || !w_scale || !w_zero || !Y) return W4A4_ERR_INVALID_ARG;
+  if (M < 1 || N < 8 || N % 8 != 0) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  w4a4_status s = check_k_group(K, group);
+  if (s != W4A4_OK) return s;
+  const size_t need = w4a8_workspace_bytes(M, K);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return W4A4_ERR_WORKSPACE;
+  int8_t* Xq = static_cast<int8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256((size_t)M * (size_t)K));
+  s = w8a8_rotate_quantize_act(X, M, K, group, Xq, xs, stream);
+  if (s != W4A4_OK) return s;
+  return w4a8_gemm(Xq, xs, Wq, w_scale, w_zero, M, N, K, group, bias, Y, nullptr, stream);
 }
 
 // ------------------------------------------------------------------ failures

@@ -69,8 +69,6 @@ constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kWaitWarp = 18;
 constexpr int kIssueBar = 2;     // named barrier: MMA warp + waiter warp
-constexpr int PS = 5;            // packed TMA stages
-constexpr int US = 6;            // widened stages
 constexpr int S8 = 5;            // INT8 TMA stages
 constexpr int LRC = 128;         // low-rank rank chunk per MMA round
 constexpr uint32_t kTmemCols = 512;
@@ -80,11 +78,19 @@ constexpr int kStageTile = 32 * 32 * 2;            // epilogue staging tile: 32 
 constexpr int kOutStageBytes = 16 * kStageTile;    // one per epilogue warp
 constexpr int kBarBytes = 512;
 
-template <bool PACKED, bool LR>
+// MODE 0: W8A8 (int8 x int8, TMA straight into the MMA layout); 1: W4A4
+// (packed INT4 x packed INT4, both widened); 2: W4A8 (int8 activations
+// copied into TMEM, packed unsigned 4-bit weights widened with their zero
+// point subtracted).
+template <int MODE, bool LR>
 struct Cfg {
+  static constexpr bool PACKED = MODE != 0;          // the widen pipeline runs
+  static constexpr int PS = MODE == 2 ? 4 : 5;       // TMA stages (A + packed B)
+  static constexpr int US = MODE == 2 ? 5 : 6;       // widened stages
   static constexpr int BN = LR ? 128 : 256;          // N per pair tile
   static constexpr int BNH = BN / 2;                 // B rows staged per CTA
-  static constexpr int kPkA = BM * BK / 2;           // packed A stage (8 KB)
+  static constexpr int kARow = MODE == 2 ? BK : BK / 2;  // bytes of an A row per k-block
+  static constexpr int kPkA = BM * kARow;            // A stage (8 KB packed, 16 KB int8)
   static constexpr int kPkB = BNH * BK / 2;
   static constexpr int kPkStage = kPkA + kPkB;
   static constexpr int kWideB = BNH * BK;            // widened B stage
@@ -92,6 +98,7 @@ struct Cfg {
   static constexpr int kI8B = BNH * BK;
   static constexpr int kI8Stage = kI8A + kI8B;
   static constexpr int kRing = PACKED ? PS * kPkStage + US * kWideB : S8 * kI8Stage;
+  static constexpr int kWOff = PS * kPkStage;        // widened B ring
   static constexpr int kLrT = BM * LRC * 2;          // T chunk: 128 rows x 128 ranks, two 64-wide boxes
   static constexpr int kLrL2 = BNH * LRC * 2;        // L2 chunk: 128 ranks x BNH columns
   static constexpr int kLrBytes = LR ? kLrT + kLrL2 : 0;
@@ -105,6 +112,8 @@ struct Cfg {
   static constexpr int kColsPerWarp = BN / 4;        // epilogue: 4 warps per TMEM lane quadrant
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kACol0 + US * (BK / 4) <= kTmemCols, "TMEM budget");
+  static_assert(PS <= 8 && US <= 8, "barrier arrays");
+  static_assert(kWOff % 1024 == 0, "128-byte swizzle atoms");
   static_assert(!LR || kLrCol + BN <= kACol0, "TMEM budget (low-rank accumulator)");
 };
 
@@ -153,15 +162,34 @@ __device__ __forceinline__ void widen16(const uint4 p, uint4& c0, uint4& c1) {
   c1.w = p.w & 0xF0F0F0F0u;
 }
 
+// 16 packed bytes (32 unsigned codes u, u_0 in the low nibble) -> 32 bytes
+// u_k - z in natural k order, as int8.  zk = 0x80808080 - z * 0x01010101:
+// each byte u + 128 - z lies in [113, 143], so the 32-bit add carries no byte
+// into the next, and flipping bit 7 turns u - z + 128 into u - z in two's
+// complement.
+__device__ __forceinline__ uint32_t sub_zero4(uint32_t x, uint32_t zk) { return (x + zk) ^ 0x80808080u; }
+__device__ __forceinline__ void widen_word_zp(uint32_t w, uint32_t zk, uint32_t& o0, uint32_t& o1) {
+  const uint32_t ev = w & 0x0F0F0F0Fu;          // u0 u2 u4 u6
+  const uint32_t od = (w >> 4) & 0x0F0F0F0Fu;   // u1 u3 u5 u7
+  o0 = sub_zero4(__byte_perm(ev, od, 0x5140), zk);  // u0 u1 u2 u3
+  o1 = sub_zero4(__byte_perm(ev, od, 0x7362), zk);  // u4 u5 u6 u7
+}
+__device__ __forceinline__ void widen16_zero_point(const uint4 p, uint32_t zk, uint4& c0, uint4& c1) {
+  widen_word_zp(p.x, zk, c0.x, c0.y);
+  widen_word_zp(p.y, zk, c0.z, c0.w);
+  widen_word_zp(p.z, zk, c1.x, c1.y);
+  widen_word_zp(p.w, zk, c1.z, c1.w);
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-// int32 accumulator -> float.  Widened products carry a factor 2^8; after the
+// int32 accumulator -> float.  W4A4 products carry a factor 2^8; after the
 // shift |t| <= 64 K <= 2^21, so t is recovered exactly from the mantissa of
 // 1.5 * 2^23 + t (two full-rate ALU operations instead of a conversion-unit
-// I2F).  The INT8 accumulator can exceed 2^22 and is rounded by I2F.
-template <bool PACKED>
+// I2F).  W8A8 and W4A8 accumulators can exceed 2^22 and are rounded by I2F.
+template <bool SHIFTED>
 __device__ __forceinline__ float acc_to_float(uint32_t v) {
-  if constexpr (PACKED) {
+  if constexpr (SHIFTED) {
     const int t = static_cast<int>(v) >> 8;
     return __fsub_rn(__int_as_float(t + 0x4B400000), 12582912.0f);
   } else {
@@ -169,16 +197,19 @@ __device__ __forceinline__ float acc_to_float(uint32_t v) {
   }
 }
 
-template <bool PACKED, bool LR>
+template <int MODE, bool LR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
                 const __grid_constant__ CUtensorMap tmL2) {
-  using C = Cfg<PACKED, LR>;
+  using C = Cfg<MODE, LR>;
+  constexpr bool PACKED = C::PACKED;
+  constexpr int PS = C::PS;
+  constexpr int US = C::US;
   constexpr int BN = C::BN;
   constexpr int BNH = C::BNH;
   const GemmArgs& p = prm.a;
-  constexpr int kShift = PACKED ? 8 : 0;  // widened products carry 2^8
+  constexpr int kShift = MODE == 1 ? 8 : 0;  // W4A4 widened products carry 2^8
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -240,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int NS = PACKED ? PS : S8;
       constexpr int kStageBytes = PACKED ? C::kPkStage : C::kI8Stage;
       constexpr int kABytes = PACKED ? C::kPkA : C::kI8A;
-      constexpr int kColBytes = PACKED ? BK / 2 : BK;
+      constexpr int kColA = PACKED ? C::kARow : BK;   // bytes per k-block of an A / B row
+      constexpr int kColB = PACKED ? BK / 2 : BK;
       int s = 0, lr_n = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -255,8 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
           mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
-          tma_load_2d(dst, &tmA, kb * kColBytes, row_a, &bar->tma_full[s]);
-          tma_load_2d(dst + kABytes, &tmB, kb * kColBytes, row_b, &bar->tma_full[s]);
+          tma_load_2d(dst, &tmA, kb * kColA, row_a, &bar->tma_full[s]);
+          tma_load_2d(dst + kABytes, &tmB, kb * kColB, row_b, &bar->tma_full[s]);
           if (++s == NS) { s = 0; ph ^= 1u; }
         }
         if (LR) {
@@ -449,11 +481,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
         return true;
       }
-      const uint32_t src = sbase + (uint32_t)(ps * C::kPkStage + (is_a ? 0 : C::kPkA) + r * (BK / 2));
-      const uint32_t rsw64 = (uint32_t)((r >> 1) & 3);
-      uint4 pk[4];
+      // A8: this thread copies an int8 activation row (128 bytes, 128-byte
+      // swizzle) into TMEM instead of widening packed codes
+      constexpr bool kA8 = MODE == 2;
+      const bool a8 = kA8 && is_a;
+      const uint32_t src = sbase + (uint32_t)(ps * C::kPkStage + (is_a ? 0 : C::kPkA) +
+                                              r * (is_a ? C::kARow : BK / 2));
+      const uint32_t rsw = a8 ? (uint32_t)(r & 7) : (uint32_t)((r >> 1) & 3);
+      uint4 pk[kA8 ? 8 : 4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw64) << 4));
+      for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw) << 4));
+      if constexpr (kA8) {
+        if (a8) {
+#pragma unroll
+          for (int c = 4; c < 8; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw) << 4));
+        } else {
+#pragma unroll
+          for (int c = 4; c < 8; ++c) pk[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       // Hand the packed stage back to TMA only once every lane's loads have
       // returned: the arrive is made data-dependent on all loaded words (an
       // mbarrier arrive by itself does not wait for this warp's outstanding
@@ -462,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // value.
       uint32_t seen = 0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) seen ^= pk[c].x ^ pk[c].y ^ pk[c].z ^ pk[c].w;
+      for (int c = 0; c < (kA8 ? 8 : 4); ++c) seen ^= pk[c].x ^ pk[c].y ^ pk[c].z ^ pk[c].w;
       seen = __reduce_or_sync(0xffffffffu, seen);
       if (lane == (seen == 0x9E3779B9u ? 1 : 0)) mbar_arrive(&bar->tma_empty[ps]);
       if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
@@ -472,12 +518,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (is_a) {
         uint32_t regs[32];
+        if constexpr (kA8) {
+          // unswizzled 16-byte chunk c of the row is stored at chunk c ^ (r & 7)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 c0, c1;
-          widen16(pk[c], c0, c1);
-          regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
-          regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
+          for (int c = 0; c < 8; ++c) {
+            regs[4 * c + 0] = pk[c].x; regs[4 * c + 1] = pk[c].y; regs[4 * c + 2] = pk[c].z; regs[4 * c + 3] = pk[c].w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 c0, c1;
+            widen16(pk[c], c0, c1);
+            regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
+            regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
+          }
         }
         tmem_st_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kACol0 + (uint32_t)(u * (BK / 4)), regs);
         tmem_wait_st();
@@ -486,10 +540,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t row =
             sbase + (uint32_t)(PS * C::kPkStage + u * C::kWideB + (r >> 3) * 1024 + (r & 7) * 128);
         const uint32_t rsw128 = (uint32_t)(r & 7);
+        uint32_t zk = 0;
+        if constexpr (kA8) {
+          // zero point of this weight row, as the per-byte bias 128 - z
+          const int n = tile_n(g / nk) + (int)rank * BNH + r;
+          const uint32_t z = n < p.N ? (uint32_t)__ldg(p.w_zero + n) : 0u;
+          zk = 0x80808080u - z * 0x01010101u;
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 c0, c1;
-          widen16(pk[c], c0, c1);
+          if constexpr (kA8)
+            widen16_zero_point(pk[c], zk, c0, c1);
+          else
+            widen16(pk[c], c0, c1);
           st_shared_v4(row + ((((uint32_t)(2 * c)) ^ rsw128) << 4), c0);
           st_shared_v4(row + ((((uint32_t)(2 * c + 1)) ^ rsw128) << 4), c1);
         }
@@ -566,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             const int jj = 4 * q + h;
-            float t = __fmul_rn(__fmul_rn(acc_to_float<PACKED>(vv[jj]), sa), wv[h]);
+            float t = __fmul_rn(__fmul_rn(acc_to_float<MODE == 1>(vv[jj]), sa), wv[h]);
             if (LR) t = __fadd_rn(t, __uint_as_float(v[1][jj]));
             y[h] = __fadd_rn(t, bv[h]);
           }
@@ -650,10 +714,10 @@ bool make_tmap(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool PACKED, bool LR>
+template <int MODE, bool LR>
 cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
-  using C = Cfg<PACKED, LR>;
-  auto kern = gemm_kernel<PACKED, LR>;
+  using C = Cfg<MODE, LR>;
+  auto kern = gemm_kernel<MODE, LR>;
   static int configured[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -664,11 +728,14 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
     configured[dev] = 1;
   }
   CUtensorMap tA, tB, tY, tT, tL2;
-  const uint64_t row_bytes = PACKED ? (uint64_t)a.K / 2 : (uint64_t)a.K;
-  const uint32_t box_cols = PACKED ? BK / 2 : BK;
-  const CUtensorMapSwizzle swz = PACKED ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.A, (uint64_t)a.M, row_bytes, box_cols, BM, swz) ||
-      !make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.B, (uint64_t)a.N, row_bytes, box_cols, C::BNH, swz) ||
+  // packed 4-bit rows: 64-byte boxes, 64-byte swizzle; int8 rows: 128-byte
+  // boxes, 128-byte swizzle
+  const bool a_packed = MODE == 1, b_packed = MODE != 0;
+  const CUtensorMapSwizzle swz64 = CU_TENSOR_MAP_SWIZZLE_64B, swz128 = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.A, (uint64_t)a.M, a_packed ? a.K / 2 : a.K,
+                 a_packed ? BK / 2 : BK, BM, a_packed ? swz64 : swz128) ||
+      !make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.B, (uint64_t)a.N, b_packed ? a.K / 2 : a.K,
+                 b_packed ? BK / 2 : BK, C::BNH, b_packed ? swz64 : swz128) ||
       !make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.Y, (uint64_t)a.M, (uint64_t)a.N, 32, 32,
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
@@ -715,11 +782,12 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
 
 unsigned int* device_error_word();
 
-cudaError_t launch_gemm(const GemmArgs& a, bool packed_int4, cudaStream_t st) {
+cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st) {
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorInvalidDevicePointer;
-  if (!packed_int4) return launch_impl<false, false>(a, err, st);
-  return a.rank > 0 ? launch_impl<true, true>(a, err, st) : launch_impl<true, false>(a, err, st);
+  if (mode == GemmMode::kW8A8) return launch_impl<0, false>(a, err, st);
+  if (mode == GemmMode::kW4A8) return launch_impl<2, false>(a, err, st);
+  return a.rank > 0 ? launch_impl<1, true>(a, err, st) : launch_impl<1, false>(a, err, st);
 }
 
 }  // namespace w4a4

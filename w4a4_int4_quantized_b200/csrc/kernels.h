@@ -6,8 +6,10 @@
 
 namespace w4a4 {
 
+// qmax 7: symmetric INT4 (packed); 127: symmetric INT8; 15: asymmetric 4-bit
+// with a zero point per row (packed unsigned codes; `zero` [rows], else null).
 cudaError_t launch_rotate_quantize(const uint16_t* X, int rows, int K, int group, int qmax, uint8_t* out,
-                                   float* scale, cudaStream_t st);
+                                   float* scale, uint8_t* zero, cudaStream_t st);
 
 struct GemmArgs {
   const uint8_t* A;        // activation codes [M, K/2] packed or [M, K] int8
@@ -22,9 +24,14 @@ struct GemmArgs {
   const uint16_t* bias;    // [N] bf16 or null
   uint16_t* Y;             // [M, N] bf16
   int32_t* acc_debug;      // [M, N] int32 or null
+  const uint8_t* w_zero;   // W4A8: zero point per weight row [N] (codes 0..15), else null
 };
 
-cudaError_t launch_gemm(const GemmArgs& a, bool packed_int4, cudaStream_t st);
+// kW4A4: packed INT4 x packed INT4 (optional low-rank); kW8A8: int8 x int8;
+// kW4A8: int8 activations x packed unsigned 4-bit weights with zero points.
+enum class GemmMode { kW8A8 = 0, kW4A4 = 1, kW4A8 = 2 };
+
+cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st);
 
 // T[M, r] (bf16) = X[M, K] (bf16) x L1[K, r] (bf16), fp32 accumulation.
 cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,

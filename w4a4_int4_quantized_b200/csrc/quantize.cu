@@ -75,9 +75,9 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // (value j of a word in bits 4j..4j+3), INT8 {.x lo, .x hi, .y lo, .y hi}.
 // The fast form brackets each quotient between two fused multiply-adds and
 // ORs any disagreement into `bad`; the exact form uses IEEE division.
-template <bool INT4, bool EXACT>
+template <bool INT4, bool EXACT, bool ASYM = false>
 __device__ __forceinline__ void quantize_block8(const float2* P8, float2 ih, float2 il, float s, uint32_t* bw,
-                                                uint32_t& bad) {
+                                                uint32_t& bad, int zoff = 0) {
   const float2 mg = make_float2(kMagic, kMagic);
   uint32_t tx[8], ty[8];
 #pragma unroll
@@ -91,6 +91,14 @@ __device__ __forceinline__ void quantize_block8(const float2* P8, float2 ih, flo
       tx[j] = __float_as_uint(th.x);
       ty[j] = __float_as_uint(th.y);
       bad |= (tx[j] ^ __float_as_uint(tl.x)) | (ty[j] ^ __float_as_uint(tl.y));
+    }
+  }
+  if (ASYM) {
+    // unsigned codes clamp(rint + z, 0, 15); zoff = z - bits(1.5 * 2^23)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      tx[j] = (uint32_t)min(max((int)tx[j] + zoff, 0), 15);
+      ty[j] = (uint32_t)min(max((int)ty[j] + zoff, 0), 15);
     }
   }
   if (INT4) {
@@ -109,15 +117,30 @@ __device__ __forceinline__ void quantize_block8(const float2* P8, float2 ih, flo
 // registers held while in flight), so the loads of the next blocks overlap
 // the rotation and quantization of the current one.  One thread owns one
 // group; its g values go from shared memory straight into float2 registers.
+// Order-preserving unsigned key of a float (for shared-memory atomic min/max).
+__device__ __forceinline__ uint32_t fkey(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float fkey_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// QMAX: 7 = symmetric INT4 (packed), 127 = symmetric INT8, 15 = asymmetric
+// 4-bit with a zero point (W4A8 weights, packed unsigned codes): per row
+// s = fl32(fl32(max - min) / 15), z = clamp(rint(fl32(-min / s)), 0, 15),
+// q = clamp(rint(fl32(y / s)) + z, 0, 15), zero point written to `zero`.
 template <int G, bool ROT, int QMAX, int MAXT>
 __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
     rotate_quantize_kernel(const uint16_t* __restrict__ X, int M, int K, int rows_per_blk, uint8_t* __restrict__ out,
-                           float* __restrict__ scale) {
+                           float* __restrict__ scale, uint8_t* __restrict__ zero) {
   constexpr int HALF = G / 2;
-  constexpr bool INT4 = (QMAX == 7);
+  constexpr bool ASYM = (QMAX == 15);
+  constexpr bool INT4 = (QMAX == 7) || ASYM;
   constexpr int GS = group_stride<G>();
   extern __shared__ __align__(16) uint8_t stage_mem[];
   __shared__ unsigned int rowmax[2][MAXT];
+  __shared__ unsigned int rowmin[ASYM ? 2 : 1][ASYM ? MAXT : 1];   // order-preserving keys (ASYM)
 
   const int gpr = K / G;
   const int tid = threadIdx.x;
@@ -143,6 +166,7 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
   };
 
   rowmax[0][tid] = 0u;
+  if (ASYM) rowmin[0][tid] = 0xFFFFFFFFu;
   // launched with programmatic stream serialization: wait for the previous
   // kernel of the stream (it may produce X, or still read this output)
   grid_dependency_wait();
@@ -156,8 +180,12 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
     cp_async_wait<kStages - 2>();
     __syncthreads();
     issue(it + kStages - 1);
-    if (tid < rows_per_blk) rowmax[(it + 1) & 1][tid] = 0u;
+    if (tid < rows_per_blk) {
+      rowmax[(it + 1) & 1][tid] = 0u;
+      if (ASYM) rowmin[(it + 1) & 1][tid] = 0xFFFFFFFFu;
+    }
     unsigned int* rmax = rowmax[it & 1];
+    unsigned int* rmin = rowmin[ASYM ? (it & 1) : 0];
 
     const long row = (long)blk * rows_per_blk + lr;
     const bool active = (lr < rows_per_blk) && (row < M);
@@ -215,13 +243,35 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
 #pragma unroll
         for (int i = 0; i < HALF; ++i) amax = max3(amax, fabsf(P[i].x), fabsf(P[i].y));
       }
-      atomicMax(&rmax[lr], __float_as_uint(amax));
+      if (ASYM) {
+        // the last stage above already wrote the outputs back into P
+        float mn = P[0].x, mx = P[0].x;
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          mn = fminf(mn, fminf(P[i].x, P[i].y));
+          mx = fmaxf(mx, fmaxf(P[i].x, P[i].y));
+        }
+        atomicMax(&rmax[lr], fkey(mx));
+        atomicMin(&rmin[lr], fkey(mn));
+      } else {
+        atomicMax(&rmax[lr], __float_as_uint(amax));
+      }
     }
     __syncthreads();
     if (!active) continue;
 
-    const float amax = __uint_as_float(rmax[lr]);
-    const float s = __fdiv_rn(amax, (float)QMAX);
+    float s;
+    int zoff = 0;
+    if (ASYM) {
+      const float mx = fkey_value(rmax[lr]), mn = fkey_value(rmin[lr]);
+      s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+      int z = 0;
+      if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
+      zoff = z - (int)__float_as_uint(kMagic);
+      if (grp == 0) zero[row] = (uint8_t)z;
+    } else {
+      s = __fdiv_rn(__uint_as_float(rmax[lr]), (float)QMAX);
+    }
     if (grp == 0) scale[row] = s;
     float inv_hi = 0.0f, inv_lo = 0.0f;
     if (s != 0.0f) {
@@ -248,8 +298,8 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
         const int blk8 = c * SB + b;
         uint32_t bw[INT4 ? 2 : 4];
         uint32_t bad = 0u;
-        quantize_block8<INT4, false>(P + 8 * blk8, ih, il, s, bw, bad);
-        if (bad) quantize_block8<INT4, true>(P + 8 * blk8, ih, il, s, bw, bad);
+        quantize_block8<INT4, false, ASYM>(P + 8 * blk8, ih, il, s, bw, bad, zoff);
+        if (bad) quantize_block8<INT4, true, ASYM>(P + 8 * blk8, ih, il, s, bw, bad, zoff);
         if (INT4) {
           w[b] = bw[0];
           w[SB + b] = bw[1];
@@ -309,7 +359,8 @@ cudaError_t pick_shape(int M, int K, int dev, RqShape& out) {
 }
 
 template <int G, bool ROT, int QMAX, int MAXT>
-cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* scale, cudaStream_t st) {
+cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* scale, uint8_t* zero,
+                        cudaStream_t st) {
   auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -346,7 +397,7 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, sh.rows_per_blk, out, scale);
+  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, sh.rows_per_blk, out, scale, zero);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -354,26 +405,30 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
 // Rows of up to 128 groups run in 128-thread CTAs (three per SM); wider rows
 // (K / g > 128) in 256-thread CTAs, one group per thread either way.
 template <int G, bool ROT, int QMAX>
-cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scale, cudaStream_t st) {
-  if (K / G <= 128) return launch_rq_t<G, ROT, QMAX, 128>(X, M, K, out, scale, st);
-  return launch_rq_t<G, ROT, QMAX, 256>(X, M, K, out, scale, st);
+cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scale, uint8_t* zero, cudaStream_t st) {
+  if (K / G <= 128) return launch_rq_t<G, ROT, QMAX, 128>(X, M, K, out, scale, zero, st);
+  return launch_rq_t<G, ROT, QMAX, 256>(X, M, K, out, scale, zero, st);
+}
+
+template <int QMAX>
+cudaError_t launch_rq_group(const uint16_t* X, int rows, int K, int group, uint8_t* out, float* scale, uint8_t* zero,
+                            cudaStream_t st) {
+  if (group == 64) return launch_rq<64, true, QMAX>(X, rows, K, out, scale, zero, st);
+  if (group == 128) return launch_rq<128, true, QMAX>(X, rows, K, out, scale, zero, st);
+  return launch_rq<128, false, QMAX>(X, rows, K, out, scale, zero, st);
 }
 
 }  // namespace
 
-// Rows of X [rows, K] bf16 -> codes (packed nibbles [rows, K/2] when qmax == 7,
-// int8 [rows, K] when qmax == 127) and one fp32 scale per row.  group 0 turns
-// the rotation off.  Shapes are validated by the caller.
+// Rows of X [rows, K] bf16 -> codes and one fp32 scale per row: packed
+// nibbles [rows, K/2] when qmax == 7 (symmetric) or qmax == 15 (asymmetric,
+// zero point per row written to `zero`), int8 [rows, K] when qmax == 127.
+// group 0 turns the rotation off.  Shapes are validated by the caller.
 cudaError_t launch_rotate_quantize(const uint16_t* X, int rows, int K, int group, int qmax, uint8_t* out,
-                                   float* scale, cudaStream_t st) {
-  if (qmax == 7) {
-    if (group == 64) return launch_rq<64, true, 7>(X, rows, K, out, scale, st);
-    if (group == 128) return launch_rq<128, true, 7>(X, rows, K, out, scale, st);
-    return launch_rq<128, false, 7>(X, rows, K, out, scale, st);
-  }
-  if (group == 64) return launch_rq<64, true, 127>(X, rows, K, out, scale, st);
-  if (group == 128) return launch_rq<128, true, 127>(X, rows, K, out, scale, st);
-  return launch_rq<128, false, 127>(X, rows, K, out, scale, st);
+                                   float* scale, uint8_t* zero, cudaStream_t st) {
+  if (qmax == 7) return launch_rq_group<7>(X, rows, K, group, out, scale, nullptr, st);
+  if (qmax == 15) return launch_rq_group<15>(X, rows, K, group, out, scale, zero, st);
+  return launch_rq_group<127>(X, rows, K, group, out, scale, nullptr, st);
 }
 
 }  // namespace w4a4
