@@ -42,8 +42,9 @@ HBM_NOMINAL_GBS = 8000.0
 # they were taken from (sha256 prefix); reported as null once the source
 # changes.
 MEASURED_TRAFFIC = {
-    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6104a6ec622ada01", 11.880192e6 + 0.009728e6),
-    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "44fa9ab62139cc24", 28.378112e6 + 512.0),
+    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "5a6b710f1ec7a816", 11.880448e6 + 0.05504e6),
+    "gemm_w4a8": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "5a6b710f1ec7a816", 18.96192e6 + 0.114176e6),
+    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "0a39f00184b08d94", 28.377856e6),
 }
 
 
@@ -146,7 +147,7 @@ def _dist_init(n_gpus: int):
     return rank, world, local
 
 
-def cpu_baseline(spec, budget_s: float = 10.0) -> dict:
+def cpu_baseline(spec, budget_s: float = 10.0, variant: str = "w4a4") -> dict:
     """The CPU oracle as it stands, on the host cores, on a bounded sample of
     the workload: the per-step path (activation rotate + quantize, integer
     GEMM, epilogue) for a subset of token rows against the full weight matrix
@@ -154,11 +155,18 @@ def cpu_baseline(spec, budget_s: float = 10.0) -> dict:
     import oracle
     from w4a4_int4_quantized_b200 import inputs
     d = inputs.make_layer(spec)
-    _, ws, wq = oracle.quantize_w4(d["W"], spec.group)
+    if variant == "w4a8":
+        _, ws, wz, wu = oracle.quantize_w4a8_weights(d["W"], spec.group)
+        wq = (wu.astype(np.int16) - wz.astype(np.int16)[:, None]).astype(np.int8)
+    else:
+        _, ws, wq = oracle.quantize_w4(d["W"], spec.group)
     rows = 8
     while True:
         t0 = time.perf_counter()
-        _, xs, xq = oracle.quantize_w4(d["X"][:rows], spec.group)
+        if variant == "w4a8":
+            xq, xs = oracle.quantize_w8(d["X"][:rows], spec.group)
+        else:
+            _, xs, xq = oracle.quantize_w4(d["X"][:rows], spec.group)
         acc = oracle.int_gemm(xq, wq)
         oracle.epilogue(acc, xs, ws, spec.group, None, None, d["bias"])
         dt = time.perf_counter() - t0
@@ -171,20 +179,28 @@ def cpu_baseline(spec, budget_s: float = 10.0) -> dict:
                       f"(act quant + int GEMM + epilogue), {dt:.1f} s"}
 
 
+def _metric_name(variant: str, spec) -> str:
+    v = variant.upper()
+    return (f"{v} linear TOPS & us/layer (M={spec.M},K={spec.K},N={spec.N}) and % of B200 INT8 TC peak"
+            if spec.name != "attn_proj" or variant != "w4a4"
+            else "W4A4 linear TOPS & us/layer (M=4608,K=N=3072) and % of B200 INT8 TC peak")
+
+
 def run_reference(args, spec):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(spec, budget_s=budget / 4)
-    vals = [cpu_baseline(spec, budget_s=budget) for _ in range(args.steps)]
+        cpu_baseline(spec, budget_s=budget / 4, variant=args.variant)
+    vals = [cpu_baseline(spec, budget_s=budget, variant=args.variant) for _ in range(args.steps)]
     v = statistics.median([b["value"] for b in vals])
     line = {
-        "impl": "reference", "metric": "W4A4 linear TOPS (M=4608, K=N=3072)", "value": v, "unit": "TOPS",
+        "impl": "reference", "metric": _metric_name(args.variant, spec), "value": v, "unit": "TOPS",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 2.0 * spec.M * spec.N * spec.K / (v * 1e12) * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes, int64 acc, f64 epilogue",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": ("int8 x 4-bit" if args.variant == "w4a8" else "int4") + " codes, int64 acc, f64 epilogue",
         "data": "synthetic", "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N,
                                         "group": spec.group, "rank": spec.rank},
         "cpu_baseline": {"value": v, "unit": "TOPS", "cores": vals[0]["cores"], "kind": "oracle",
@@ -204,12 +220,17 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--variant", choices=["w4a4", "w4a8"], default="w4a4",
+                    help="w4a8: rotated int8 activations x zero-pointed 4-bit weights")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
     from w4a4_int4_quantized_b200 import inputs
     spec = inputs.WORKLOADS[args.workload]
+    w4a8 = args.variant == "w4a8"
+    if w4a8 and spec.rank:
+        raise SystemExit("the W4A8 path has no low-rank branch: pick a workload with rank 0")
     if args.impl == "reference":
         run_reference(args, spec)
         return
@@ -234,10 +255,14 @@ def main():
     for i in range(args.sets):
         d = inputs.make_layer(spec, seed_offset=1000 * rank + i)
         X = dev(d["X"])
-        Wq, ws = w4.w4a4_quantize_weights(dev(d["W"]), g)
-        s = dict(X=X, Wq=Wq, ws=ws, bias=dev(d["bias"]) if d["bias"] is not None else None,
+        if w4a8:
+            Wq, ws, wz = w4.w4a8_quantize_weights(dev(d["W"]), g)
+        else:
+            (Wq, ws), wz = w4.w4a4_quantize_weights(dev(d["W"]), g), None
+        s = dict(X=X, Wq=Wq, ws=ws, wz=wz, bias=dev(d["bias"]) if d["bias"] is not None else None,
                  L1=dev(d["L1"]) if r else None, L2=dev(d["L2"]) if r else None,
-                 Xq=torch.empty((M, K // 2), dtype=torch.uint8, device="cuda"),
+                 Xq=(torch.empty((M, K), dtype=torch.int8, device="cuda") if w4a8 else
+                     torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")),
                  xs=torch.empty((M,), dtype=torch.float32, device="cuda"),
                  T=torch.empty((M, r), dtype=torch.bfloat16, device="cuda") if r else None,
                  Y=torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
@@ -245,9 +270,22 @@ def main():
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
+    def k1(s):
+        if w4a8:
+            w4.w8a8_rotate_quantize_act(s["X"], g, Xq=s["Xq"], x_scale=s["xs"], stream=stream)
+        else:
+            w4.w4a4_rotate_quantize_act(s["X"], g, s["L1"], Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=stream)
+
+    def k2(s):
+        if w4a8:
+            w4.w4a8_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], s["wz"], g, s["bias"], Y=s["Y"], stream=stream)
+        else:
+            w4.w4a4_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], g, s["T"], s["L2"], s["bias"], Y=s["Y"],
+                         stream=stream)
+
     def step(s):
-        w4.w4a4_rotate_quantize_act(s["X"], g, s["L1"], Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=stream)
-        w4.w4a4_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], g, s["T"], s["L2"], s["bias"], Y=s["Y"], stream=stream)
+        k1(s)
+        k2(s)
 
     for i in range(args.warmup):
         step(sets[i % len(sets)])
@@ -291,10 +329,8 @@ def main():
         return a.elapsed_time(b) / n
 
     n_split = min(args.steps, 200)
-    k1_ms = timed(lambda s: w4.w4a4_rotate_quantize_act(s["X"], g, s["L1"], Xq=s["Xq"], x_scale=s["xs"],
-                                                         T=s["T"], stream=stream), n_split)
-    k2_ms = timed(lambda s: w4.w4a4_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], g, s["T"], s["L2"], s["bias"],
-                                         Y=s["Y"], stream=stream), n_split)
+    k1_ms = timed(k1, n_split)
+    k2_ms = timed(k2, n_split)
     err = w4.w4a4_get_device_error()
     if err:
         raise SystemExit(f"device error word {err:#x}")
@@ -310,17 +346,26 @@ def main():
         hx = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
         hx.copy_(s["X"].cpu())
         hy = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
-        ws_buf = torch.empty((w4.w4a4_workspace_bytes(M, K, r),), dtype=torch.uint8, device="cuda")
+        ws_buf = torch.empty((w4.w4a8_workspace_bytes(M, K) if w4a8 else w4.w4a4_workspace_bytes(M, K, r),),
+                             dtype=torch.uint8, device="cuda")
+
+        def linear():
+            if w4a8:
+                w4.w4a8_linear(s["X"], s["Wq"], s["ws"], s["wz"], g, s["bias"], Y=s["Y"], workspace=ws_buf)
+            else:
+                w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"],
+                               workspace=ws_buf)
+
         for _ in range(3):
             s["X"].copy_(hx, non_blocking=True)
-            w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"], workspace=ws_buf)
+            linear()
             hy.copy_(s["Y"], non_blocking=True)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
             s["X"].copy_(hx, non_blocking=True)
-            w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"], workspace=ws_buf)
+            linear()
             hy.copy_(s["Y"], non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -334,29 +379,31 @@ def main():
         k2 = k2_ms
         k2_tops = ops / (k2 * 1e-3) / 1e12
         int8_peak = 2.0 * pk["bf16_sustained"]   # nominal int8 : bf16 ratio is 2
-        k1_bytes = M * K * 2 + M * K // 2 + M * 4
+        k1_bytes = M * K * 2 + (M * K if w4a8 else M * K // 2) + M * 4
         line = {
-            "metric": "W4A4 linear TOPS & us/layer (M=4608,K=N=3072) and % of B200 INT8 TC peak",
+            "metric": _metric_name(args.variant, spec),
             "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "us_per_layer": total_ms / args.steps * 1e3,
             "frac_of_int8_nominal_peak": value / INT8_NOMINAL_TOPS,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int4 codes (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
-            "config": {"workload": spec.name, "M": M, "K": K, "N": N, "group": g, "rank": r,
+            "dtype": ("int8 activations x 4-bit zero-pointed weights" if w4a8 else "int4 codes")
+                     + " (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
+            "config": {"workload": spec.name, "variant": args.variant, "M": M, "K": K, "N": N, "group": g, "rank": r,
                        "bias": spec.bias, "parallelism": f"replicas x{world} (token shards, no exchange)",
                        "l2": f"{args.sets} rotating input sets (> L2)"},
             "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3, "note": "each kernel timed alone, back to back"},
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
-                         "frac": k2_tops / int8_peak, "traffic": _traffic("gemm", spec.name),
+                         "frac": k2_tops / int8_peak,
+                         "traffic": _traffic("gemm_w4a8" if w4a8 else "gemm", spec.name),
                          "peak_note": f"int8 = 2 x {pk['source']} sustained bf16 {pk['bf16_sustained']} TFLOP/s"},
             "roofline_k1": {"bound": "hbm", "achieved": k1_bytes / (k1 * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": k1_bytes / (k1 * 1e-3) / 1e9 / pk["hbm_gbs"],
-                            "traffic": _traffic("rotate_quantize", spec.name)},
+                            "traffic": None if w4a8 else _traffic("rotate_quantize", spec.name)},
             "gpu_launches": 2 * args.steps + (args.steps if r else 0),
             "clocks": clk, "wall_s": wall, "e2e": e2e,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(spec)
+            line["cpu_baseline"] = cpu_baseline(spec, variant=args.variant)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -79,14 +79,14 @@ constexpr int kOutStageBytes = 16 * kStageTile;    // one per epilogue warp
 constexpr int kBarBytes = 512;
 
 // MODE 0: W8A8 (int8 x int8, TMA straight into the MMA layout); 1: W4A4
-// (packed INT4 x packed INT4, both widened); 2: W4A8 (int8 activations
-// copied into TMEM, packed unsigned 4-bit weights widened with their zero
-// point subtracted).
+// (packed INT4 x packed INT4, both widened, A into TMEM); 2: W4A8 (the int8
+// activation tile is read by the MMA straight from its TMA stage; packed
+// unsigned 4-bit weights are widened with their zero point subtracted).
 template <int MODE, bool LR>
 struct Cfg {
   static constexpr bool PACKED = MODE != 0;          // the widen pipeline runs
-  static constexpr int PS = MODE == 2 ? 4 : 5;       // TMA stages (A + packed B)
-  static constexpr int US = MODE == 2 ? 5 : 6;       // widened stages
+  static constexpr int PS = 5;                      // TMA stages (A + packed B)
+  static constexpr int US = MODE == 2 ? 4 : 6;       // widened stages (W4A8: B only)
   static constexpr int BN = LR ? 128 : 256;          // N per pair tile
   static constexpr int BNH = BN / 2;                 // B rows staged per CTA
   static constexpr int kARow = MODE == 2 ? BK : BK / 2;  // bytes of an A row per k-block
@@ -241,7 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int s = 0; s < 8; ++s) {
         mbar_init(&bar->tma_full[s], 1);
-        mbar_init(&bar->tma_empty[s], PACKED ? 8 : 1);
+        // W4A4: the 8 widen warps of a set read the stage; W4A8: its 4 B
+        // warps plus the MMA commit (the MMA reads A from the stage); W8A8:
+        // the MMA commit
+        mbar_init(&bar->tma_empty[s], MODE == 1 ? 8 : (MODE == 2 ? 5 : 1));
         mbar_init(&bar->full[s], PACKED ? 16 : 1);  // 8 widen warps per CTA, or 1 relay
         mbar_init(&bar->empty[s], 1);
       }
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
       constexpr uint32_t idesc_lr = idesc_bf16(2 * BM, BN, false, true);
       constexpr int NS = PACKED ? US : S8;
-      int s = 0;
+      int s = 0, ps = 0;   // widened / TMA stage of the k-block
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
         for (int kb = 0; kb < nk; ++kb) {
@@ -358,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           if (lane == 0) {
-            if (PACKED) {
+            if (MODE == 1) {
               const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
 #pragma unroll
               for (int ks = 0; ks < BK / 32; ++ks)
@@ -366,6 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
                                (kb | ks) != 0 ? 1u : 0u);
               tc_commit_pair_mc(&bar->empty[s], 0x3);
+            } else if (MODE == 2) {
+              const uint32_t a_stage = sbase + (uint32_t)(ps * C::kPkStage);
+              const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
+#pragma unroll
+              for (int ks = 0; ks < BK / 32; ++ks)
+                mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
+                               smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
+                               (kb | ks) != 0 ? 1u : 0u);
+              tc_commit_pair_mc(&bar->empty[s], 0x3);
+              tc_commit_pair_mc(&bar->tma_empty[ps], 0x3);
             } else {
               const uint32_t a_stage = sbase + (uint32_t)(s * C::kI8Stage);
 #pragma unroll
@@ -378,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (++s == NS) s = 0;
+          if (++ps == PS) ps = 0;
         }
         if (LR) {
           // T L2 into the fp32 accumulator: A = T (K-major, 128-byte
@@ -481,25 +495,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
         return true;
       }
-      // A8: this thread copies an int8 activation row (128 bytes, 128-byte
-      // swizzle) into TMEM instead of widening packed codes
       constexpr bool kA8 = MODE == 2;
-      const bool a8 = kA8 && is_a;
-      const uint32_t src = sbase + (uint32_t)(ps * C::kPkStage + (is_a ? 0 : C::kPkA) +
-                                              r * (is_a ? C::kARow : BK / 2));
-      const uint32_t rsw = a8 ? (uint32_t)(r & 7) : (uint32_t)((r >> 1) & 3);
-      uint4 pk[kA8 ? 8 : 4];
+      if (kA8 && is_a) {
+        // W4A8: the MMA reads this int8 A tile straight from the TMA stage
+        // (released by its commit); the A warps only report, after the
+        // previous use of widened stage u has been consumed, that the tile
+        // has landed in this CTA
+        if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
+          set_device_error(prm.err, kDevErrTimeoutEmpty);
+          return false;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
+        return true;
+      }
+      const uint32_t src = sbase + (uint32_t)(ps * C::kPkStage + (is_a ? 0 : C::kPkA) + r * (BK / 2));
+      const uint32_t rsw = (uint32_t)((r >> 1) & 3);
+      uint4 pk[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw) << 4));
-      if constexpr (kA8) {
-        if (a8) {
-#pragma unroll
-          for (int c = 4; c < 8; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw) << 4));
-        } else {
-#pragma unroll
-          for (int c = 4; c < 8; ++c) pk[c] = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
       // Hand the packed stage back to TMA only once every lane's loads have
       // returned: the arrive is made data-dependent on all loaded words (an
       // mbarrier arrive by itself does not wait for this warp's outstanding
@@ -508,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // value.
       uint32_t seen = 0;
 #pragma unroll
-      for (int c = 0; c < (kA8 ? 8 : 4); ++c) seen ^= pk[c].x ^ pk[c].y ^ pk[c].z ^ pk[c].w;
+      for (int c = 0; c < 4; ++c) seen ^= pk[c].x ^ pk[c].y ^ pk[c].z ^ pk[c].w;
       seen = __reduce_or_sync(0xffffffffu, seen);
       if (lane == (seen == 0x9E3779B9u ? 1 : 0)) mbar_arrive(&bar->tma_empty[ps]);
       if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
@@ -518,20 +532,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (is_a) {
         uint32_t regs[32];
-        if constexpr (kA8) {
-          // unswizzled 16-byte chunk c of the row is stored at chunk c ^ (r & 7)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            regs[4 * c + 0] = pk[c].x; regs[4 * c + 1] = pk[c].y; regs[4 * c + 2] = pk[c].z; regs[4 * c + 3] = pk[c].w;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 c0, c1;
-            widen16(pk[c], c0, c1);
-            regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
-            regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
-          }
+        for (int c = 0; c < 4; ++c) {
+          uint4 c0, c1;
+          widen16(pk[c], c0, c1);
+          regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
+          regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
         }
         tmem_st_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kACol0 + (uint32_t)(u * (BK / 4)), regs);
         tmem_wait_st();
