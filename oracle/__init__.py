@@ -58,6 +58,7 @@ def _load():
         lib.oracle_epilogue.argtypes = [P, P, P, L, L, I, P, P, I, P, P]
         lib.oracle_f32_to_bf16.argtypes = [P, L, P]
         lib.oracle_f64_to_bf16.argtypes = [P, L, P]
+        lib.oracle_lora_merge.argtypes = [P, P, I, P, P, I, ctypes.c_float, I, I, P, P]
         _lib = lib
     return _lib
 
@@ -246,6 +247,35 @@ def linear_w4a8(X, W, g, bias=None):
     acc = int_gemm(xq, centered)
     Y = epilogue(acc, xs, ws, g, None, None, bias)
     return dict(x_q=xq, x_scale=xs, w_packed=wp, w_scale=ws, w_zero=wz, w_q=wq, acc=acc, Y=Y)
+
+
+def lora_merge(L1, L2, A, B, scale: float):
+    """Low-rank operands of the merged branch: ([L1 | A], [L2 ; bf16(scale * B)])."""
+    A = _bf16(A)
+    B = _bf16(B)
+    K, rl = A.shape
+    N = B.shape[1]
+    r = 0 if L1 is None else L1.shape[1]
+    L1 = _bf16(L1) if r else np.zeros((K, 0), np.uint16)
+    L2 = _bf16(L2) if r else np.zeros((0, N), np.uint16)
+    L1o = np.empty((K, r + rl), dtype=np.uint16)
+    L2o = np.empty((r + rl, N), dtype=np.uint16)
+    _load().oracle_lora_merge(_ptr(L1) if r else None, _ptr(L2) if r else None, r, _ptr(A), _ptr(B), rl,
+                              float(scale), K, N, _ptr(L1o), _ptr(L2o))
+    return L1o, L2o
+
+
+def linear_w4a4_lora(X, W, g, L1, L2, A, B, scale: float, bias=None):
+    """W4A4 layer with the SVDQuant branch and a runtime LoRA beside it:
+    Y = dequant(acc) + (X L1) L2 + scale (X A) B + bias, the low-rank terms in
+    fp64 from the bf16 operands (unmerged)."""
+    base = linear_w4a4(X, W, g, L1, L2, bias)
+    TA = lowrank_down(X, A)
+    lora = float(np.float32(scale)) * (TA @ bf16_to_f64(B))
+    out = dict(base)
+    out["Y"] = base["Y"] + lora
+    out["T_lora"] = TA
+    return out
 
 
 def linear_w8a8(X, W, g, bias=None):

@@ -283,6 +283,25 @@ void oracle_lowrank_down(const uint16_t *X, const uint16_t *L1, long M, int K, i
         }
 }
 
+/* Runtime LoRA merged into the low-rank branch ("ComfyUI-INT4-Fast",
+   "INT4 Quantized Inference Comes to ComfyUI": LoRAs apply on top of the 4-bit
+   layer; "Krea 2 Turbo - SVDQuant", "What's included": the low-rank branch
+   runs beside the 4-bit product).  L1o = [L1 | A] ([K, r + rl]),
+   L2o = [L2 ; bf16(fl32(scale * B))] ([r + rl, N]): the LoRA's scale is folded
+   into its up matrix with one fp32 multiply and one round-to-nearest-even
+   narrowing per element. */
+void oracle_lora_merge(const uint16_t *L1, const uint16_t *L2, int r, const uint16_t *A, const uint16_t *B, int rl,
+                       float scale, int K, int N, uint16_t *L1o, uint16_t *L2o) {
+    const int rt = r + rl;
+    for (int k = 0; k < K; ++k)
+        for (int j = 0; j < rt; ++j)
+            L1o[(long)k * rt + j] = j < r ? L1[(long)k * r + j] : A[(long)k * rl + (j - r)];
+    for (int j = 0; j < rt; ++j)
+        for (int n = 0; n < N; ++n)
+            L2o[(long)j * N + n] = j < r ? L2[(long)j * N + n]
+                                         : f32_to_bf16(scale * bf16_to_f32(B[(long)(j - r) * N + n]));
+}
+
 /* Y[m][n] = ((acc * sa[m]) * sw[n]) * (1/g) + sum_j T[m][j] * L2[j][n] + bias[n]
    in fp64.  g == 0 means no rotation (factor 1).  T/L2 are ignored when r == 0;
    bias may be NULL. */

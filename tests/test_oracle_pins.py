@@ -19,6 +19,9 @@ textbook facts, library routines, closed forms and hand-derived fixtures):
     code 0, maximum -> 14/15, exact zero -> zero point, monotone codes, error
     bound; centered integer product recomputed with NumPy int64; lower error
     than W4A4 on the same layer.
+  * Runtime LoRA: merged operands are the inputs concatenated, the scaled
+    block equals torch's bf16 narrowing of NumPy's fp32 product; with W = 0
+    the layer is (X L1) L2 + s (X A) B + b in NumPy fp64, merged or not.
   * Planted mistakes (in copies of oracle outputs, on the CPU) are caught.
 """
 from __future__ import annotations
@@ -452,3 +455,60 @@ def test_w4a8_pins_catch_planted_mistakes():
     t = (y[0] / s).astype(np.float32)
     away = (np.sign(t) * np.floor(np.abs(t) + 0.5)).astype(np.int64) + zz
     assert away.tolist() != codes
+
+
+# ---------------------------------------------------------------- runtime LoRA merged into the low-rank branch
+def _lora_operands(K=256, N=96, r=16, rl=32, seed=40):
+    rng = np.random.default_rng(seed)
+    L1 = _bf16(rng.standard_normal((K, r), dtype=np.float32) * 0.05)
+    L2 = _bf16(rng.standard_normal((r, N), dtype=np.float32) * 0.05)
+    A = _bf16(rng.standard_normal((K, rl), dtype=np.float32) * 0.05)
+    B = _bf16(rng.standard_normal((rl, N), dtype=np.float32) * 0.05)
+    return L1, L2, A, B
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.5, 4.0, 0.3, 1.7])
+def test_lora_merge_concatenates_and_scales(scale):
+    """[L1 | A] and [L2 ; bf16(fl32(scale B))]: the copied blocks are the
+    inputs; a power-of-two scale is exact; otherwise the scaled entries are
+    torch's bf16 narrowing of NumPy's fp32 product, within one bf16 ulp of the
+    exact product."""
+    torch = pytest.importorskip("torch")
+    L1, L2, A, B = _lora_operands()
+    L1o, L2o = oracle.lora_merge(L1, L2, A, B, scale)
+    assert np.array_equal(L1o[:, :16], L1) and np.array_equal(L1o[:, 16:], A)
+    assert np.array_equal(L2o[:16], L2)
+    exact = np.float64(np.float32(scale)) * oracle.bf16_to_f64(B)
+    got = oracle.bf16_to_f64(L2o[16:])
+    if scale in (1.0, 0.5, 4.0):
+        assert np.array_equal(got, exact)
+    prod32 = np.float32(scale) * _f32(B)
+    ref = torch.from_numpy(prod32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(L2o[16:], ref)
+    assert np.all(np.abs(got - exact) <= 2.0 ** -8 * np.abs(exact))
+
+
+def test_lora_layer_reduces_to_two_matmuls_when_weights_vanish():
+    """W = 0: Y = (X L1) L2 + s (X A) B + b, a NumPy fp64 product; the merged
+    operands give the same branch (exact for a power-of-two scale); s = 0
+    leaves the plain W4A4 layer."""
+    K, N, M = 256, 96, 12
+    L1, L2, A, B = _lora_operands(K, N)
+    rng = np.random.default_rng(41)
+    X = _bf16(rng.standard_normal((M, K), dtype=np.float32))
+    W = np.zeros((N, K), np.uint16)
+    b = _bf16(rng.standard_normal(N, dtype=np.float32) * 0.01)
+    f = oracle.bf16_to_f64
+    ref = (f(X) @ f(L1)) @ f(L2) + 0.5 * ((f(X) @ f(A)) @ f(B)) + f(b)
+    got = oracle.linear_w4a4_lora(X, W, 64, L1, L2, A, B, 0.5, b)["Y"]
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+    L1o, L2o = oracle.lora_merge(L1, L2, A, B, 0.5)
+    merged = (f(X) @ f(L1o)) @ f(L2o) + f(b)
+    assert np.allclose(merged, ref, rtol=1e-12, atol=1e-12)
+    Wn = _bf16(rng.standard_normal((N, K), dtype=np.float32) * 0.02)
+    plain = oracle.linear_w4a4(X, Wn, 64, L1, L2, b)["Y"]
+    assert np.array_equal(oracle.linear_w4a4_lora(X, Wn, 64, L1, L2, A, B, 0.0, b)["Y"], plain)
+    # planted mistakes: the scale applied twice, or A and B taken from the
+    # SVDQuant pair, fail the reduction
+    assert not np.allclose(ref + 0.5 * ((f(X) @ f(A)) @ f(B)), got, rtol=1e-6)
+    assert not np.allclose((f(X) @ f(L1)) @ f(L2) * 1.5 + f(b), got, rtol=1e-6)
