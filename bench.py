@@ -220,6 +220,8 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--lora", type=int, default=0,
+                    help="rank of a runtime LoRA merged beside the layer's low-rank branch (w4a4)")
     ap.add_argument("--variant", choices=["w4a4", "w4a8"], default="w4a4",
                     help="w4a8: rotated int8 activations x zero-pointed 4-bit weights")
     args = ap.parse_args()
@@ -229,8 +231,8 @@ def main():
     from w4a4_int4_quantized_b200 import inputs
     spec = inputs.WORKLOADS[args.workload]
     w4a8 = args.variant == "w4a8"
-    if w4a8 and spec.rank:
-        raise SystemExit("the W4A8 path has no low-rank branch: pick a workload with rank 0")
+    if w4a8 and (spec.rank or args.lora):
+        raise SystemExit("the W4A8 path has no low-rank branch: pick a workload with rank 0 and no --lora")
     if args.impl == "reference":
         run_reference(args, spec)
         return
@@ -246,7 +248,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     w4.load_library()
-    g, M, K, N, r = spec.group, spec.M, spec.K, spec.N, spec.rank
+    g, M, K, N, r = spec.group, spec.M, spec.K, spec.N, spec.rank + args.lora
 
     def dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
@@ -259,8 +261,15 @@ def main():
             Wq, ws, wz = w4.w4a8_quantize_weights(dev(d["W"]), g)
         else:
             (Wq, ws), wz = w4.w4a4_quantize_weights(dev(d["W"]), g), None
+        L1 = dev(d["L1"]) if spec.rank else None
+        L2 = dev(d["L2"]) if spec.rank else None
+        if args.lora:
+            # runtime LoRA (A, B ~ N(0, 0.01), scale 1) merged into one branch
+            A = dev(inputs.random_bf16((K, args.lora), seed=7000 + i, std=0.01))
+            B = dev(inputs.random_bf16((args.lora, N), seed=8000 + i, std=0.01))
+            L1, L2 = w4.w4a4_lora_merge(L1, L2, A, B, 1.0)
         s = dict(X=X, Wq=Wq, ws=ws, wz=wz, bias=dev(d["bias"]) if d["bias"] is not None else None,
-                 L1=dev(d["L1"]) if r else None, L2=dev(d["L2"]) if r else None,
+                 L1=L1, L2=L2,
                  Xq=(torch.empty((M, K), dtype=torch.int8, device="cuda") if w4a8 else
                      torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")),
                  xs=torch.empty((M,), dtype=torch.float32, device="cuda"),
@@ -389,6 +398,7 @@ def main():
             "dtype": ("int8 activations x 4-bit zero-pointed weights" if w4a8 else "int4 codes")
                      + " (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
             "config": {"workload": spec.name, "variant": args.variant, "M": M, "K": K, "N": N, "group": g, "rank": r,
+                       "lora_rank": args.lora,
                        "bias": spec.bias, "parallelism": f"replicas x{world} (token shards, no exchange)",
                        "l2": f"{args.sets} rotating input sets (> L2)"},
             "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3, "note": "each kernel timed alone, back to back"},

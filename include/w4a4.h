@@ -206,6 +206,27 @@ w4a4_status w4a8_linear(const void* X, const uint8_t* Wq, const float* w_scale, 
                         int N, int K, int group, const void* bias, void* Y, void* workspace,
                         size_t workspace_bytes, w4a4_stream_t stream);
 
+/* ---------------------------------------------------------------- runtime LoRA */
+/* A LoRA applied at run time beside the SVDQuant low-rank branch ("ComfyUI-
+ * INT4-Fast", "INT4 Quantized Inference Comes to ComfyUI": LoRAs on top of
+ * the 4-bit layers; "Krea 2 Turbo - SVDQuant", "What's included": the
+ * low-rank branch beside the 4-bit product).  Writes the operands of one
+ * combined branch of rank r + lora_rank:
+ *   L1_out [K, r + lora_rank] = [L1 | A]            (bf16, row-major)
+ *   L2_out [r + lora_rank, N] = [L2 ; bf16(fl32(lora_scale * B))]
+ * so that w4a4_rotate_quantize_act / w4a4_gemm / w4a4_linear with these
+ * operands and rank r + lora_rank compute
+ *   dequant(acc) + (X L1) L2 + lora_scale (X A) B + bias
+ * with a single epilogue low-rank MMA.  L1 [K, r], L2 [r, N] (may be NULL
+ * when r == 0), A [K, lora_rank], B [lora_rank, N]: bf16, caller-owned
+ * device memory, 16-byte aligned.  Shapes: r % 16 == 0, lora_rank >= 16 and
+ * lora_rank % 16 == 0, r + lora_rank <= 256, N % 8 == 0.  Asynchronous on
+ * `stream`; the outputs must not alias the inputs.  The pages give no
+ * formula for the merge; this is the plainest reading (the scale folded into
+ * the up matrix). */
+w4a4_status w4a4_lora_merge(const void* L1, const void* L2, int rank, const void* A, const void* B, int lora_rank,
+                            float lora_scale, int K, int N, void* L1_out, void* L2_out, w4a4_stream_t stream);
+
 /* ---------------------------------------------------------------- failures */
 /* Kernels never trap: a wait on another part of the kernel that runs past its
  * time limit (2 s) records a code in a per-device error word and lets the

@@ -46,7 +46,7 @@ def test_header_declares_the_documented_entry_points():
               "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
               "w4a4_workspace_bytes", "w8a8_workspace_bytes", "w4a4_status_string", "w4a4_version",
               "w4a4_get_device_error", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear",
-              "w4a8_workspace_bytes"]:
+              "w4a8_workspace_bytes", "w4a4_lora_merge"]:
         assert n in names
 
 
@@ -107,6 +107,24 @@ def test_gemm_validation(lib):
     bad = list(args); bad[13] = ODD                    # misaligned debug output
     assert f(*bad) == MISALIGNED
     assert lib.w8a8_gemm(A, B, C, D, 64, 4, 256, 128, NUL, E, NUL, NUL) == SHAPE
+
+
+def test_lora_merge_validation(lib):
+    f = lib.w4a4_lora_merge
+    args = [A, B, 16, C, D, 32, 0.5, 256, 512, E, E, NUL]
+    bad = list(args); bad[3] = NUL                      # no LoRA down matrix
+    assert f(*bad) == INVALID
+    bad = list(args); bad[0] = NUL                      # rank > 0 without L1
+    assert f(*bad) == INVALID
+    bad = list(args); bad[5] = 8                        # LoRA rank not a multiple of 16
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[5] = 256                      # combined rank above 256
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[8] = 12                       # N not a multiple of 8
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[9] = ODD
+    assert f(*bad) == MISALIGNED
+    assert f(NUL, NUL, 0, C, D, 32, 0.5, 256, 512, ODD, E, NUL) == MISALIGNED   # r = 0 needs no L1 / L2
 
 
 def test_w4a8_validation(lib):

@@ -228,6 +228,40 @@ def test_w4a8_layer_parity(M, N, K, g):
     assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
 
 
+@pytest.mark.parametrize("r,rl,scale", [(0, 32, 1.0), (16, 32, 0.3), (64, 64, 1.7)])
+def test_lora_merge_bitexact(r, rl, scale):
+    import torch
+    K, N = 640, 264
+    L1 = inputs.random_bf16((K, r), seed=1, std=0.05) if r else None
+    L2 = inputs.random_bf16((r, N), seed=2, std=0.05) if r else None
+    A = inputs.random_bf16((K, rl), seed=3, std=0.05)
+    B = inputs.random_bf16((rl, N), seed=4, std=0.05)
+    L1o, L2o = w4.w4a4_lora_merge(dev_bf16(L1) if r else None, dev_bf16(L2) if r else None,
+                                  dev_bf16(A), dev_bf16(B), scale)
+    ref1, ref2 = oracle.lora_merge(L1, L2, A, B, scale)
+    assert np.array_equal(L1o.cpu().view(torch.int16).numpy().view(np.uint16), ref1)
+    assert np.array_equal(L2o.cpu().view(torch.int16).numpy().view(np.uint16), ref2)
+
+
+@pytest.mark.parametrize("M,N,K,g,r,rl,scale", [(130, 520, 1280, 64, 32, 16, 0.7), (257, 768, 3072, 128, 0, 64, 1.0),
+                                                 (96, 512, 12288, 128, 128, 128, 0.25)])
+def test_w4a4_layer_with_runtime_lora(M, N, K, g, r, rl, scale):
+    """The merged operands in the unchanged W4A4 path give the layer with the
+    LoRA beside the SVDQuant branch (oracle: unmerged, fp64)."""
+    import torch
+    d = _layer(M, N, K, g, r, True, seed=M + N + K + rl)
+    A = inputs.random_bf16((K, rl), seed=M + 5, std=0.01)
+    B = inputs.random_bf16((rl, N), seed=N + 6, std=0.01)
+    ref = oracle.linear_w4a4_lora(d["X"], d["W"], g, d["L1"], d["L2"], A, B, scale, d["bias"])
+    X, W, b = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    Wq, ws = w4.w4a4_quantize_weights(W, g)
+    L1m, L2m = w4.w4a4_lora_merge(dev_bf16(d["L1"]) if r else None, dev_bf16(d["L2"]) if r else None,
+                                  dev_bf16(A), dev_bf16(B), scale)
+    Y = w4.w4a4_linear(X, Wq, ws, g, L1m, L2m, b)
+    torch.cuda.synchronize()
+    check_output(host_f64(Y), ref["Y"], lowrank=True)
+
+
 def test_attn_proj_full_size_sampled():
     """The attention-projection workload at full size (M=4608, K=N=3072,
     g=128, bias), in the launch configuration the benchmark times

@@ -22,7 +22,7 @@ __all__ = [
     "w4a4_workspace_bytes", "w4a4_linear_noalloc", "NOALLOC_SCRATCH_BYTES",
     "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
     "w8a8_workspace_bytes", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear", "w4a8_workspace_bytes",
-    "w4a4_get_device_error",
+    "w4a4_lora_merge", "w4a4_get_device_error",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -74,6 +74,7 @@ def load_library():
         "w4a8_gemm": ([P, P, P, P, P, I, I, I, I, P, P, P, P], S),
         "w4a8_workspace_bytes": ([I, I], Z),
         "w4a8_linear": ([P, P, P, P, I, I, I, I, P, P, P, Z, P], S),
+        "w4a4_lora_merge": ([P, P, I, P, P, I, ctypes.c_float, I, I, P, P, P], S),
         "w4a4_get_device_error": ([P, ctypes.POINTER(ctypes.c_uint)], S),
     }
     for name, (args, res) in sig.items():
@@ -277,6 +278,21 @@ def w4a8_linear(X, Wq, w_scale, w_zero, group, bias=None, Y=None, workspace=None
         _ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(w_zero), M, N, K, group, _ptr(bias), _ptr(Y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return Y
+
+
+def w4a4_lora_merge(L1, L2, A, B, lora_scale: float, L1_out=None, L2_out=None, stream=None):
+    """Operands of the combined low-rank branch: ([L1 | A], [L2 ; bf16(scale B)]).
+    L1 / L2 may be None (no SVDQuant branch)."""
+    import torch
+    K, rl = A.shape
+    N = B.shape[1]
+    r = 0 if L1 is None else L1.shape[1]
+    L1_out = _empty((K, r + rl), torch.bfloat16, A) if L1_out is None else L1_out
+    L2_out = _empty((r + rl, N), torch.bfloat16, A) if L2_out is None else L2_out
+    _check("w4a4_lora_merge", load_library().w4a4_lora_merge(
+        _ptr(L1), _ptr(L2), r, _ptr(A), _ptr(B), rl, float(lora_scale), K, N, _ptr(L1_out), _ptr(L2_out),
+        _stream(stream)))
+    return L1_out, L2_out
 
 
 def w4a4_get_device_error(stream=None) -> int:

@@ -280,6 +280,25 @@ w4a4_status w4a8_linear(const void* X, const uint8_t* Wq, const float* w_scale, 
   return w4a8_gemm(Xq, xs, Wq, w_scale, w_zero, M, N, K, group, bias, Y, nullptr, stream);
 }
 
+// ------------------------------------------------------------------ runtime LoRA
+w4a4_status w4a4_lora_merge(const void* L1, const void* L2, int rank, const void* A, const void* B, int lora_rank,
+                            float lora_scale, int K, int N, void* L1_out, void* L2_out, w4a4_stream_t stream) {
+  if (!A || !B || !L1_out || !L2_out) return W4A4_ERR_INVALID_ARG;
+  if (rank > 0 && (!L1 || !L2)) return W4A4_ERR_INVALID_ARG;
+  if (rank < 0 || rank % 16 != 0 || lora_rank < 16 || lora_rank % 16 != 0 || rank + lora_rank > 256)
+    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if (K < 1 || N < 8 || N % 8 != 0) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if ((rank > 0 && (!aligned16(L1) || !aligned16(L2))) || !aligned16(A) || !aligned16(B) || !aligned16(L1_out) ||
+      !aligned16(L2_out))
+    return W4A4_ERR_MISALIGNED;
+  w4a4_status s = check_device();
+  if (s != W4A4_OK) return s;
+  return cuda_status(launch_lora_merge(static_cast<const uint16_t*>(L1), static_cast<const uint16_t*>(L2), rank,
+                                       static_cast<const uint16_t*>(A), static_cast<const uint16_t*>(B), lora_rank,
+                                       lora_scale, K, N, static_cast<uint16_t*>(L1_out),
+                                       static_cast<uint16_t*>(L2_out), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------------------------ failures
 w4a4_status w4a4_get_device_error(w4a4_stream_t stream, unsigned int* code) {
   w4a4_status s = check_device();

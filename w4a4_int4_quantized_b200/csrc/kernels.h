@@ -37,4 +37,8 @@ cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st);
 cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
                                 cudaStream_t st);
 
+// [L1 | A] and [L2 ; bf16(fl32(scale * B))] (rank r + rl low-rank operands).
+cudaError_t launch_lora_merge(const uint16_t* L1, const uint16_t* L2, int r, const uint16_t* A, const uint16_t* B,
+                              int rl, float scale, int K, int N, uint16_t* L1o, uint16_t* L2o, cudaStream_t st);
+
 }  // namespace w4a4
