@@ -59,6 +59,7 @@ def _load():
         lib.oracle_f32_to_bf16.argtypes = [P, L, P]
         lib.oracle_f64_to_bf16.argtypes = [P, L, P]
         lib.oracle_lora_merge.argtypes = [P, P, I, P, P, I, ctypes.c_float, I, I, P, P]
+        lib.oracle_gelu_tanh.argtypes = [P, L, P]
         _lib = lib
     return _lib
 
@@ -247,6 +248,24 @@ def linear_w4a8(X, W, g, bias=None):
     acc = int_gemm(xq, centered)
     Y = epilogue(acc, xs, ws, g, None, None, bias)
     return dict(x_q=xq, x_scale=xs, w_packed=wp, w_scale=ws, w_zero=wz, w_q=wq, acc=acc, Y=Y)
+
+
+def gelu_tanh(x: np.ndarray) -> np.ndarray:
+    """GELU, tanh approximation, in fp64."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    _load().oracle_gelu_tanh(_ptr(x), x.size, _ptr(y))
+    return y
+
+
+def linear_w4a4_gelu(X, W, g, L1=None, L2=None, bias=None):
+    """W4A4 layer followed by GELU(tanh) on its unrounded output (fp64): the
+    fused up-projection of the MLP."""
+    out = linear_w4a4(X, W, g, L1, L2, bias)
+    out = dict(out)
+    out["Y_linear"] = out["Y"]
+    out["Y"] = gelu_tanh(out["Y"])
+    return out
 
 
 def lora_merge(L1, L2, A, B, scale: float):

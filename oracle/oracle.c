@@ -283,6 +283,20 @@ void oracle_lowrank_down(const uint16_t *X, const uint16_t *L1, long M, int K, i
         }
 }
 
+/* GELU with the tanh approximation, in fp64 (the MLP between the up and down
+   projections of the pages' diffusion transformer blocks, "Load Diffusion
+   Model INT4 (W4A4)": every linear layer of the model runs in 4 bit, the
+   activation between them in high precision):
+   gelu(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))). */
+void oracle_gelu_tanh(const double *x, long n, double *y) {
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    #pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i) {
+        const double v = x[i];
+        y[i] = 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+    }
+}
+
 /* Runtime LoRA merged into the low-rank branch ("ComfyUI-INT4-Fast",
    "INT4 Quantized Inference Comes to ComfyUI": LoRAs apply on top of the 4-bit
    layer; "Krea 2 Turbo - SVDQuant", "What's included": the low-rank branch

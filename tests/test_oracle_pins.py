@@ -22,6 +22,8 @@ textbook facts, library routines, closed forms and hand-derived fixtures):
   * Runtime LoRA: merged operands are the inputs concatenated, the scaled
     block equals torch's bf16 narrowing of NumPy's fp32 product; with W = 0
     the layer is (X L1) L2 + s (X A) B + b in NumPy fp64, merged or not.
+  * GELU(tanh): torch's tanh-approximate GELU in fp64; gelu(0) = 0,
+    gelu(x) - gelu(-x) = x; the fused layer is GELU of the unrounded output.
   * Planted mistakes (in copies of oracle outputs, on the CPU) are caught.
 """
 from __future__ import annotations
@@ -512,3 +514,30 @@ def test_lora_layer_reduces_to_two_matmuls_when_weights_vanish():
     # SVDQuant pair, fail the reduction
     assert not np.allclose(ref + 0.5 * ((f(X) @ f(A)) @ f(B)), got, rtol=1e-6)
     assert not np.allclose((f(X) @ f(L1)) @ f(L2) * 1.5 + f(b), got, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- GELU (fused MLP up-projection)
+def test_gelu_matches_torch_and_identities():
+    """fp64 GELU(tanh) equals torch's tanh-approximate GELU in fp64; exact
+    identities: gelu(0) = 0 and gelu(x) - gelu(-x) = x; limits x and 0."""
+    torch = pytest.importorskip("torch")
+    x = np.random.default_rng(50).standard_normal(20000) * 4.0
+    y = oracle.gelu_tanh(x)
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    assert np.max(np.abs(y - ref)) <= 1e-14 * np.max(np.abs(x))
+    assert oracle.gelu_tanh(np.zeros(3))[0] == 0.0
+    assert np.max(np.abs((y - oracle.gelu_tanh(-x)) - x)) <= 1e-13 * np.max(np.abs(x))
+    big = np.array([30.0, -30.0])
+    assert np.allclose(oracle.gelu_tanh(big), [30.0, 0.0], atol=1e-12)
+    # planted mistake: the erf form differs from the tanh form by > 1e-4
+    erf_form = torch.nn.functional.gelu(torch.from_numpy(x)).numpy()
+    assert np.max(np.abs(erf_form - y)) > 1e-4
+
+
+def test_gelu_layer_applies_after_the_epilogue():
+    spec = inputs.LayerSpec("gl", 16, 256, 64, 64, rank=16, bias=True, seed=51, outlier_scale=10.0)
+    d = inputs.make_layer(spec)
+    out = oracle.linear_w4a4_gelu(d["X"], d["W"], 64, d["L1"], d["L2"], d["bias"])
+    base = oracle.linear_w4a4(d["X"], d["W"], 64, d["L1"], d["L2"], d["bias"])
+    assert np.array_equal(out["Y_linear"], base["Y"])
+    assert np.array_equal(out["Y"], oracle.gelu_tanh(base["Y"]))
