@@ -210,6 +210,93 @@ def run_reference(args, spec):
     print(json.dumps(line), flush=True)
 
 
+def run_mlp(args):
+    """The MLP pair at M = 4608 (3072 -> 12288 -> 3072, r = 128 on both, g = 128)
+    with GELU fused into the up-projection epilogue: per step rotate+quantize
+    X, low-rank down, up GEMM with GELU, rotate+quantize h, low-rank down,
+    down GEMM.  Also times the unfused chain (plain up GEMM, torch GELU on
+    [M, 12288] bf16, same down layer) for comparison.  Single GPU."""
+    import torch
+    import w4a4_int4_quantized_b200 as w4
+    from w4a4_int4_quantized_b200 import inputs
+    w4.load_library()
+    su, sd = inputs.WORKLOADS["mlp_up"], inputs.WORKLOADS["mlp_down"]
+    M, D, H, g, r = su.M, su.K, su.N, su.group, su.rank
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    du, dd = inputs.make_layer(su), inputs.make_layer(sd)
+    Wq_u, ws_u = w4.w4a4_quantize_weights(dev(du["W"]), g)
+    Wq_d, ws_d = w4.w4a4_quantize_weights(dev(dd["W"]), g)
+    L1u, L2u, bu = dev(du["L1"]), dev(du["L2"]), dev(du["bias"])
+    L1d, L2d, bd = dev(dd["L1"]), dev(dd["L2"]), dev(dd["bias"])
+    sets = []
+    for i in range(2):
+        X = dev(inputs.make_layer(su, seed_offset=i)["X"])
+        sets.append(dict(X=X, Xq=torch.empty((M, D // 2), dtype=torch.uint8, device="cuda"),
+                         xs=torch.empty((M,), dtype=torch.float32, device="cuda"),
+                         T=torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
+                         h=torch.empty((M, H), dtype=torch.bfloat16, device="cuda"),
+                         hq=torch.empty((M, H // 2), dtype=torch.uint8, device="cuda"),
+                         hs=torch.empty((M,), dtype=torch.float32, device="cuda"),
+                         Th=torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
+                         Y=torch.empty((M, D), dtype=torch.bfloat16, device="cuda")))
+    stream = torch.cuda.current_stream()
+
+    def step(s, fused=True):
+        w4.w4a4_rotate_quantize_act(s["X"], g, L1u, Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=stream)
+        if fused:
+            w4.w4a4_gemm_gelu(s["Xq"], s["xs"], Wq_u, ws_u, g, s["T"], L2u, bu, Y=s["h"], stream=stream)
+        else:
+            w4.w4a4_gemm(s["Xq"], s["xs"], Wq_u, ws_u, g, s["T"], L2u, bu, Y=s["h"], stream=stream)
+            s["h"].copy_(torch.nn.functional.gelu(s["h"], approximate="tanh"))
+        w4.w4a4_rotate_quantize_act(s["h"], g, L1d, Xq=s["hq"], x_scale=s["hs"], T=s["Th"], stream=stream)
+        w4.w4a4_gemm(s["hq"], s["hs"], Wq_d, ws_d, g, s["Th"], L2d, bd, Y=s["Y"], stream=stream)
+
+    def timed(fused, n):
+        for i in range(args.warmup):
+            step(sets[i % 2], fused)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            step(sets[i % 2], fused)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = time.perf_counter()
+    ms = timed(True, args.steps)
+    clocks.mark(t0, time.perf_counter())
+    clk = clocks.stop()
+    ms_unfused = timed(False, args.steps)
+    err = w4.w4a4_get_device_error()
+    if err:
+        raise SystemExit(f"device error word {err:#x}")
+    ops = 2.0 * 2.0 * M * D * H
+    lr_flops = 2.0 * 2.0 * M * r * (D + H)
+    pk = _peaks()
+    line = {
+        "metric": "W4A4 fused MLP pair TOPS & us (M=4608, 3072->12288->3072, r=128, GELU in the up epilogue)",
+        "value": ops / (ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_mlp": ms * 1e3, "us_per_mlp_unfused": ms_unfused * 1e3,
+        "lowrank_gflop_per_step": lr_flops / 1e9,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 codes (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
+        "config": {"workload": "mlp_pair", "M": M, "D": D, "H": H, "group": g, "rank": r,
+                   "l2": "2 rotating input sets; [M, 12288] intermediates exceed L2"},
+        "roofline": {"bound": "tensor", "achieved": ops / (ms * 1e-3) / 1e12, "peak": 2.0 * pk["bf16_sustained"],
+                     "unit": "TOPS", "frac": ops / (ms * 1e-3) / 1e12 / (2.0 * pk["bf16_sustained"]),
+                     "traffic": None, "peak_note": "whole chain against the int8 tensor peak"},
+        "gpu_launches": 6 * args.steps, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -220,6 +307,8 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--mlp", action="store_true",
+                    help="time the fused MLP pair (up with GELU in its epilogue, then down) instead")
     ap.add_argument("--lora", type=int, default=0,
                     help="rank of a runtime LoRA merged beside the layer's low-rank branch (w4a4)")
     ap.add_argument("--variant", choices=["w4a4", "w4a8"], default="w4a4",
@@ -229,6 +318,12 @@ def main():
         raise SystemExit("--warmup must be >= 3")
 
     from w4a4_int4_quantized_b200 import inputs
+    if args.mlp:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the MLP chain is measured by the GPU arm only"}))
+            return
+        run_mlp(args)
+        return
     spec = inputs.WORKLOADS[args.workload]
     w4a8 = args.variant == "w4a8"
     if w4a8 and (spec.rank or args.lora):

@@ -206,6 +206,38 @@ w4a4_status w4a8_linear(const void* X, const uint8_t* Wq, const float* w_scale, 
                         int N, int K, int group, const void* bias, void* Y, void* workspace,
                         size_t workspace_bytes, w4a4_stream_t stream);
 
+/* ---------------------------------------------------------------- fused MLP */
+/* The MLP of the pages' transformer blocks runs both projections in 4 bit
+ * ("Load Diffusion Model INT4 (W4A4)", intro and "The part that actually
+ * matters: mixed precision": every linear layer goes to 4 bit, the
+ * activation between them stays in high precision).  GELU with the tanh
+ * approximation is applied in the up-projection's epilogue, on the fp32
+ * result after the bias and before the bf16 store:
+ *   gelu(y) = 0.5 y (1 + tanhf(sqrt(2/pi) (y + 0.044715 y^3))),
+ * so the down-projection's rotate + quantize reads the activated tensor
+ * directly (no separate activation pass over [M, H]).
+ * w4a4_gemm_gelu / w4a4_linear_gelu: as w4a4_gemm / w4a4_linear with the
+ * fused activation.  w4a4_mlp: Y [M, D] = linear_down(gelu(linear_up(X))) for
+ * X [M, D] bf16, up weights Wq_up [H, D/2] (+ scales, low-rank rank_up), down
+ * weights Wq_down [D, H/2] (rank_down), one rotation group for both layers;
+ * the workspace (w4a4_mlp_workspace_bytes, 256-byte aligned) holds both
+ * layers' codes and scales, their low-rank T and the activated [M, H] bf16
+ * tensor.  Shape and alignment rules are those of w4a4_linear for each
+ * layer (D and H in the K and N roles); the first failing check's status is
+ * returned. */
+w4a4_status w4a4_gemm_gelu(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale,
+                           int M, int N, int K, int group, const void* T, const void* L2, int rank, const void* bias,
+                           void* Y, int32_t* acc_debug, w4a4_stream_t stream);
+w4a4_status w4a4_linear_gelu(const void* X, const uint8_t* Wq, const float* w_scale, int M, int N, int K,
+                             int group, const void* L1, const void* L2, int rank, const void* bias, void* Y,
+                             void* workspace, size_t workspace_bytes, w4a4_stream_t stream);
+size_t w4a4_mlp_workspace_bytes(int M, int D, int H, int rank_up, int rank_down);
+w4a4_status w4a4_mlp(const void* X, int M, int D, int H, int group, const uint8_t* Wq_up, const float* w_scale_up,
+                     const void* L1_up, const void* L2_up, int rank_up, const void* bias_up, const uint8_t* Wq_down,
+                     const float* w_scale_down, const void* L1_down, const void* L2_down, int rank_down,
+                     const void* bias_down, void* Y, void* workspace, size_t workspace_bytes,
+                     w4a4_stream_t stream);
+
 /* ---------------------------------------------------------------- runtime LoRA */
 /* A LoRA applied at run time beside the SVDQuant low-rank branch ("ComfyUI-
  * INT4-Fast", "INT4 Quantized Inference Comes to ComfyUI": LoRAs on top of

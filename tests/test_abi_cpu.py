@@ -46,7 +46,8 @@ def test_header_declares_the_documented_entry_points():
               "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
               "w4a4_workspace_bytes", "w8a8_workspace_bytes", "w4a4_status_string", "w4a4_version",
               "w4a4_get_device_error", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear",
-              "w4a8_workspace_bytes", "w4a4_lora_merge"]:
+              "w4a8_workspace_bytes", "w4a4_lora_merge", "w4a4_gemm_gelu", "w4a4_linear_gelu", "w4a4_mlp",
+              "w4a4_mlp_workspace_bytes"]:
         assert n in names
 
 
@@ -107,6 +108,27 @@ def test_gemm_validation(lib):
     bad = list(args); bad[13] = ODD                    # misaligned debug output
     assert f(*bad) == MISALIGNED
     assert lib.w8a8_gemm(A, B, C, D, 64, 4, 256, 128, NUL, E, NUL, NUL) == SHAPE
+
+
+def test_mlp_workspace_and_validation(lib):
+    M, D, H = 4608, 3072, 12288
+    need = lib.w4a4_mlp_workspace_bytes(M, D, H, 128, 128)
+    up = lib.w4a4_workspace_bytes(M, D, 128)
+    down = lib.w4a4_workspace_bytes(M, H, 128)
+    assert need == up + M * H * 2 + down      # every part already 256-aligned here
+    assert lib.w4a4_mlp_workspace_bytes(0, D, H, 0, 0) == 0
+    f = lib.w4a4_mlp
+    args = [A, 64, 256, 512, 128, B, C, NUL, NUL, 0, NUL, D, E, NUL, NUL, 0, NUL, E, E,
+            lib.w4a4_mlp_workspace_bytes(64, 256, 512, 0, 0), NUL]
+    bad = list(args); bad[5] = NUL                       # no up weights
+    assert f(*bad) == INVALID
+    bad = list(args); bad[19] = 1                         # workspace too small
+    assert f(*bad) == WORKSPACE
+    bad = list(args); bad[0] = 0                          # no input  (NULL)
+    assert f(*bad) == INVALID
+    g = lib.w4a4_gemm_gelu
+    assert g(A, B, C, D, 64, 12, 256, 64, NUL, NUL, 0, NUL, E, NUL, NUL) == SHAPE
+    assert lib.w4a4_linear_gelu(A, B, C, 64, 256, 256, 64, NUL, NUL, 0, NUL, D, E, 1, NUL) == WORKSPACE
 
 
 def test_lora_merge_validation(lib):

@@ -262,6 +262,60 @@ def test_w4a4_layer_with_runtime_lora(M, N, K, g, r, rl, scale):
     check_output(host_f64(Y), ref["Y"], lowrank=True)
 
 
+@pytest.mark.parametrize("M,N,K,g,r", [(130, 520, 1280, 64, 32), (257, 768, 3072, 128, 0)])
+def test_w4a4_layer_with_fused_gelu(M, N, K, g, r):
+    """GELU(tanh) fused into the epilogue: the same accumulators, GELU of the
+    unrounded output within the layer tolerance, and the fused call equal to
+    the two-step path."""
+    import torch
+    d = _layer(M, N, K, g, r, True, seed=M + N + K + 9)
+    ref = oracle.linear_w4a4_gelu(d["X"], d["W"], g, d["L1"], d["L2"], d["bias"])
+    X, W, b = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    L1 = dev_bf16(d["L1"]) if r else None
+    L2 = dev_bf16(d["L2"]) if r else None
+    Wq, ws = w4.w4a4_quantize_weights(W, g)
+    Xq, xs, T = w4.w4a4_rotate_quantize_act(X, g, L1)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    Y = w4.w4a4_gemm_gelu(Xq, xs, Wq, ws, g, T, L2, b, acc_debug=acc)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    check_output(host_f64(Y), ref["Y"], lowrank=r > 0)
+    Y2 = w4.w4a4_linear_gelu(X, Wq, ws, g, L1, L2, b)
+    torch.cuda.synchronize()
+    assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+
+
+def test_fused_mlp_chain():
+    """w4a4_mlp = down(gelu(up(X))): its activated tensor is the fused
+    up-projection (checked against the fp64 oracle), and its output equals the
+    down-projection layer applied to that tensor (bit for bit), which in turn
+    matches the oracle fed the same bf16 tensor."""
+    import torch
+    M, D, H, g, r = 200, 512, 1536, 128, 32
+    rng = np.random.default_rng(77)
+    spec_up = inputs.LayerSpec("up", M, D, H, g, rank=r, bias=True, seed=78, outlier_scale=50.0)
+    du = inputs.make_layer(spec_up)
+    Wd = inputs.random_bf16((D, H), seed=79, std=0.02)
+    L1d = inputs.random_bf16((H, r), seed=80, std=0.01)
+    L2d = inputs.random_bf16((r, D), seed=81, std=0.01)
+    bd = inputs.random_bf16((D,), seed=82, std=0.01)
+    X = dev_bf16(du["X"])
+    Wq_u, ws_u = w4.w4a4_quantize_weights(dev_bf16(du["W"]), g)
+    Wq_d, ws_d = w4.w4a4_quantize_weights(dev_bf16(Wd), g)
+    up = dict(Wq=Wq_u, w_scale=ws_u, L1=dev_bf16(du["L1"]), L2=dev_bf16(du["L2"]), bias=dev_bf16(du["bias"]))
+    down = dict(Wq=Wq_d, w_scale=ws_d, L1=dev_bf16(L1d), L2=dev_bf16(L2d), bias=dev_bf16(bd))
+    Y = w4.w4a4_mlp(X, g, up, down)
+    h = w4.w4a4_linear_gelu(X, Wq_u, ws_u, g, up["L1"], up["L2"], up["bias"])
+    Y2 = w4.w4a4_linear(h, Wq_d, ws_d, g, down["L1"], down["L2"], down["bias"])
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    ref_h = oracle.linear_w4a4_gelu(du["X"], du["W"], g, du["L1"], du["L2"], du["bias"])
+    check_output(host_f64(h), ref_h["Y"], lowrank=True)
+    h_bits = h.cpu().view(torch.int16).numpy().view(np.uint16)
+    ref_y = oracle.linear_w4a4(h_bits, Wd, g, L1d, L2d, bd)
+    check_output(host_f64(Y), ref_y["Y"], lowrank=True)
+
+
 def test_attn_proj_full_size_sampled():
     """The attention-projection workload at full size (M=4608, K=N=3072,
     g=128, bias), in the launch configuration the benchmark times

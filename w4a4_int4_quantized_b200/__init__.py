@@ -22,7 +22,8 @@ __all__ = [
     "w4a4_workspace_bytes", "w4a4_linear_noalloc", "NOALLOC_SCRATCH_BYTES",
     "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
     "w8a8_workspace_bytes", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear", "w4a8_workspace_bytes",
-    "w4a4_lora_merge", "w4a4_get_device_error",
+    "w4a4_lora_merge", "w4a4_gemm_gelu", "w4a4_linear_gelu", "w4a4_mlp", "w4a4_mlp_workspace_bytes",
+    "w4a4_get_device_error",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -75,6 +76,10 @@ def load_library():
         "w4a8_workspace_bytes": ([I, I], Z),
         "w4a8_linear": ([P, P, P, P, I, I, I, I, P, P, P, Z, P], S),
         "w4a4_lora_merge": ([P, P, I, P, P, I, ctypes.c_float, I, I, P, P, P], S),
+        "w4a4_gemm_gelu": ([P, P, P, P, I, I, I, I, P, P, I, P, P, P, P], S),
+        "w4a4_linear_gelu": ([P, P, P, I, I, I, I, P, P, I, P, P, P, Z, P], S),
+        "w4a4_mlp_workspace_bytes": ([I, I, I, I, I], Z),
+        "w4a4_mlp": ([P, I, I, I, I, P, P, P, P, I, P, P, P, P, P, I, P, P, P, Z, P], S),
         "w4a4_get_device_error": ([P, ctypes.POINTER(ctypes.c_uint)], S),
     }
     for name, (args, res) in sig.items():
@@ -293,6 +298,61 @@ def w4a4_lora_merge(L1, L2, A, B, lora_scale: float, L1_out=None, L2_out=None, s
         _ptr(L1), _ptr(L2), r, _ptr(A), _ptr(B), rl, float(lora_scale), K, N, _ptr(L1_out), _ptr(L2_out),
         _stream(stream)))
     return L1_out, L2_out
+
+
+def w4a4_gemm_gelu(Xq, x_scale, Wq, w_scale, group, T=None, L2=None, bias=None, Y=None, acc_debug=None,
+                   stream=None):
+    """w4a4_gemm with GELU (tanh approximation) fused into the epilogue."""
+    import torch
+    M = Xq.shape[0]
+    N, Kh = Wq.shape
+    K = 2 * Kh
+    rank = 0 if T is None else T.shape[1]
+    Y = _empty((M, N), torch.bfloat16, Xq) if Y is None else Y
+    _check("w4a4_gemm_gelu", load_library().w4a4_gemm_gelu(
+        _ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, group, _ptr(T), _ptr(L2), rank, _ptr(bias),
+        _ptr(Y), _ptr(acc_debug), _stream(stream)))
+    return Y
+
+
+def w4a4_linear_gelu(X, Wq, w_scale, group, L1=None, L2=None, bias=None, Y=None, workspace=None, stream=None):
+    """w4a4_linear with GELU (tanh approximation) fused into the epilogue."""
+    import torch
+    M, K = X.shape
+    N = Wq.shape[0]
+    rank = 0 if L1 is None else L1.shape[1]
+    need = w4a4_workspace_bytes(M, K, rank)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=X.device)
+    Y = _empty((M, N), torch.bfloat16, X) if Y is None else Y
+    _check("w4a4_linear_gelu", load_library().w4a4_linear_gelu(
+        _ptr(X), _ptr(Wq), _ptr(w_scale), M, N, K, group, _ptr(L1), _ptr(L2), rank, _ptr(bias), _ptr(Y),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return Y
+
+
+def w4a4_mlp_workspace_bytes(M: int, D: int, H: int, rank_up: int, rank_down: int) -> int:
+    return int(load_library().w4a4_mlp_workspace_bytes(M, D, H, rank_up, rank_down))
+
+
+def w4a4_mlp(X, group, up, down, Y=None, workspace=None, stream=None):
+    """Y = down(gelu(up(X))).  up / down: dicts with Wq, w_scale and optional
+    L1, L2, bias (the two layers' quantized weights and low-rank operands)."""
+    import torch
+    M, D = X.shape
+    H = up["Wq"].shape[0]
+    ru = 0 if up.get("L1") is None else up["L1"].shape[1]
+    rd = 0 if down.get("L1") is None else down["L1"].shape[1]
+    need = w4a4_mlp_workspace_bytes(M, D, H, ru, rd)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    Y = _empty((M, D), torch.bfloat16, X) if Y is None else Y
+    _check("w4a4_mlp", load_library().w4a4_mlp(
+        _ptr(X), M, D, H, group, _ptr(up["Wq"]), _ptr(up["w_scale"]), _ptr(up.get("L1")), _ptr(up.get("L2")), ru,
+        _ptr(up.get("bias")), _ptr(down["Wq"]), _ptr(down["w_scale"]), _ptr(down.get("L1")),
+        _ptr(down.get("L2")), rd, _ptr(down.get("bias")), _ptr(Y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return Y
 
 
 def w4a4_get_device_error(stream=None) -> int:

@@ -158,7 +158,7 @@ w4a4_status w4a4_rotate_quantize_act(const void* X, int M, int K, int group, uin
 static w4a4_status gemm_common(const void* Xq, const float* x_scale, const void* Wq, const float* w_scale,
                                const uint8_t* w_zero, int M, int N, int K, int group, const void* T, const void* L2,
                                int rank, const void* bias, void* Y, int32_t* acc_debug, GemmMode mode,
-                               w4a4_stream_t stream) {
+                               w4a4_stream_t stream, int act = 0) {
   if (!Xq || !x_scale || !Wq || !w_scale || !Y) return W4A4_ERR_INVALID_ARG;
   if (mode == GemmMode::kW4A8 && !w_zero) return W4A4_ERR_INVALID_ARG;
   w4a4_status s = check_rank(rank);
@@ -190,6 +190,7 @@ static w4a4_status gemm_common(const void* Xq, const float* x_scale, const void*
   a.Y = static_cast<uint16_t*>(Y);
   a.acc_debug = acc_debug;
   a.w_zero = w_zero;
+  a.act = act;
   return cuda_status(launch_gemm(a, mode, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -198,6 +199,13 @@ w4a4_status w4a4_gemm(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq
                       int32_t* acc_debug, w4a4_stream_t stream) {
   return gemm_common(Xq, x_scale, Wq, w_scale, nullptr, M, N, K, group, T, L2, rank, bias, Y, acc_debug,
                      GemmMode::kW4A4, stream);
+}
+
+w4a4_status w4a4_gemm_gelu(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale,
+                           int M, int N, int K, int group, const void* T, const void* L2, int rank, const void* bias,
+                           void* Y, int32_t* acc_debug, w4a4_stream_t stream) {
+  return gemm_common(Xq, x_scale, Wq, w_scale, nullptr, M, N, K, group, T, L2, rank, bias, Y, acc_debug,
+                     GemmMode::kW4A4, stream, 1);
 }
 
 w4a4_status w8a8_gemm(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale, int M,
@@ -246,6 +254,53 @@ w4a4_status w4a4_linear(const void* X, const uint8_t* Wq, const float* w_scale, 
   s = w4a4_rotate_quantize_act(X, M, K, group, Xq, xs, L1, rank, T, stream);
   if (s != W4A4_OK) return s;
   return w4a4_gemm(Xq, xs, Wq, w_scale, M, N, K, group, T, L2, rank, bias, Y, nullptr, stream);
+}
+
+w4a4_status w4a4_linear_gelu(const void* X, const uint8_t* Wq, const float* w_scale, int M, int N, int K,
+                             int group, const void* L1, const void* L2, int rank, const void* bias, void* Y,
+                             void* workspace, size_t workspace_bytes, w4a4_stream_t stream) {
+  if (!X || !Wq || !w_scale || !Y) return W4A4_ERR_INVALID_ARG;
+  w4a4_status s = check_rank(rank);
+  if (s != W4A4_OK) return s;
+  if (rank > 0 && (!L1 || !L2)) return W4A4_ERR_INVALID_ARG;
+  if (M < 1 || N < 8 || N % 8 != 0) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if ((s = check_k_group(K, group)) != W4A4_OK) return s;
+  const size_t need = w4a4_workspace_bytes(M, K, rank);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return W4A4_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* Xq = ws;
+  float* xs = reinterpret_cast<float*>(ws + round256((size_t)M * (size_t)(K / 2)));
+  void* T = rank > 0 ? static_cast<void*>(ws + round256((size_t)M * (size_t)(K / 2)) + round256((size_t)M * 4u))
+                     : nullptr;
+  s = w4a4_rotate_quantize_act(X, M, K, group, Xq, xs, L1, rank, T, stream);
+  if (s != W4A4_OK) return s;
+  return w4a4_gemm_gelu(Xq, xs, Wq, w_scale, M, N, K, group, T, L2, rank, bias, Y, nullptr, stream);
+}
+
+size_t w4a4_mlp_workspace_bytes(int M, int D, int H, int rank_up, int rank_down) {
+  if (M < 1 || D < 2 || H < 2 || rank_up < 0 || rank_down < 0) return 0;
+  return round256(w4a4_workspace_bytes(M, D, rank_up)) + round256((size_t)M * (size_t)H * 2u) +
+         round256(w4a4_workspace_bytes(M, H, rank_down));
+}
+
+w4a4_status w4a4_mlp(const void* X, int M, int D, int H, int group, const uint8_t* Wq_up, const float* w_scale_up,
+                     const void* L1_up, const void* L2_up, int rank_up, const void* bias_up, const uint8_t* Wq_down,
+                     const float* w_scale_down, const void* L1_down, const void* L2_down, int rank_down,
+                     const void* bias_down, void* Y, void* workspace, size_t workspace_bytes,
+                     w4a4_stream_t stream) {
+  if (!X || !Wq_up || !w_scale_up || !Wq_down || !w_scale_down || !Y) return W4A4_ERR_INVALID_ARG;
+  const size_t need = w4a4_mlp_workspace_bytes(M, D, H, rank_up, rank_down);
+  if (need == 0) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return W4A4_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t up_bytes = round256(w4a4_workspace_bytes(M, D, rank_up));
+  void* h = ws + up_bytes;
+  uint8_t* ws_down = ws + up_bytes + round256((size_t)M * (size_t)H * 2u);
+  w4a4_status s = w4a4_linear_gelu(X, Wq_up, w_scale_up, M, H, D, group, L1_up, L2_up, rank_up, bias_up, h, ws,
+                                   up_bytes, stream);
+  if (s != W4A4_OK) return s;
+  return w4a4_linear(h, Wq_down, w_scale_down, M, D, H, group, L1_down, L2_down, rank_down, bias_down, Y, ws_down,
+                     round256(w4a4_workspace_bytes(M, H, rank_down)), stream);
 }
 
 w4a4_status w8a8_linear(const void* X, const int8_t* Wq, const float* w_scale, int M, int N, int K, int group,

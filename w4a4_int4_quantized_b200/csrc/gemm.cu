@@ -197,7 +197,14 @@ __device__ __forceinline__ float acc_to_float(uint32_t v) {
   }
 }
 
-template <int MODE, bool LR>
+// GELU with the tanh approximation (fused MLP up-projection), fp32.
+__device__ __forceinline__ float gelu_tanh(float x) {
+  const float c = 0.7978845608028654f;   // sqrt(2 / pi)
+  const float u = c * (x + 0.044715f * (x * x * x));
+  return 0.5f * x * (1.0f + tanhf(u));
+}
+
+template <int MODE, bool LR, bool ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
@@ -639,6 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float t = __fmul_rn(__fmul_rn(acc_to_float<MODE == 1>(vv[jj]), sa), wv[h]);
             if (LR) t = __fadd_rn(t, __uint_as_float(v[1][jj]));
             y[h] = __fadd_rn(t, bv[h]);
+            if constexpr (ACT) y[h] = gelu_tanh(y[h]);
           }
           __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
           __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
@@ -720,10 +728,10 @@ bool make_tmap(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* b
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, bool LR>
+template <int MODE, bool LR, bool ACT = false>
 cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   using C = Cfg<MODE, LR>;
-  auto kern = gemm_kernel<MODE, LR>;
+  auto kern = gemm_kernel<MODE, LR, ACT>;
   static int configured[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -793,6 +801,8 @@ cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st) {
   if (!err) return cudaErrorInvalidDevicePointer;
   if (mode == GemmMode::kW8A8) return launch_impl<0, false>(a, err, st);
   if (mode == GemmMode::kW4A8) return launch_impl<2, false>(a, err, st);
+  if (a.act == 1)
+    return a.rank > 0 ? launch_impl<1, true, true>(a, err, st) : launch_impl<1, false, true>(a, err, st);
   return a.rank > 0 ? launch_impl<1, true>(a, err, st) : launch_impl<1, false>(a, err, st);
 }
 

@@ -25,6 +25,7 @@ struct GemmArgs {
   uint16_t* Y;             // [M, N] bf16
   int32_t* acc_debug;      // [M, N] int32 or null
   const uint8_t* w_zero;   // W4A8: zero point per weight row [N] (codes 0..15), else null
+  int act;                 // W4A4: 0 none, 1 GELU (tanh approximation) applied before the bf16 store
 };
 
 // kW4A4: packed INT4 x packed INT4 (optional low-rank); kW8A8: int8 x int8;
