@@ -60,6 +60,10 @@ def _load():
         lib.oracle_f64_to_bf16.argtypes = [P, L, P]
         lib.oracle_lora_merge.argtypes = [P, P, I, P, P, I, ctypes.c_float, I, I, P, P]
         lib.oracle_gelu_tanh.argtypes = [P, L, P]
+        lib.oracle_philox4x64.argtypes = [P, P, P]
+        lib.oracle_sr_uniform.argtypes = [L, ctypes.c_uint64, P]
+        lib.oracle_lora_bake.argtypes = [P, P, P, I, I, I, ctypes.c_float, P]
+        lib.oracle_quantize_sr.argtypes = [P, L, I, P, P, P]
         _lib = lib
     return _lib
 
@@ -248,6 +252,51 @@ def linear_w4a8(X, W, g, bias=None):
     acc = int_gemm(xq, centered)
     Y = epilogue(acc, xs, ws, g, None, None, bias)
     return dict(x_q=xq, x_scale=xs, w_packed=wp, w_scale=ws, w_zero=wz, w_q=wq, acc=acc, Y=Y)
+
+
+def philox4x64(counter, key) -> np.ndarray:
+    """Philox4x64-10 block for a 4-word counter and 2-word key (uint64)."""
+    c = np.ascontiguousarray(counter, dtype=np.uint64)
+    k = np.ascontiguousarray(key, dtype=np.uint64)
+    out = np.empty(4, dtype=np.uint64)
+    _load().oracle_philox4x64(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def sr_uniform(n: int, seed: int) -> np.ndarray:
+    """The u in [0, 1) of elements 0..n-1 of a row-major array (fp32)."""
+    u = np.empty(n, dtype=np.float32)
+    _load().oracle_sr_uniform(n, seed, _ptr(u))
+    return u
+
+
+def lora_bake(W, A, B, scale: float) -> np.ndarray:
+    """bf16(W + scale * (A @ B)^T), fp32 index-order FMA sums."""
+    W, A, B = _bf16(W), _bf16(A), _bf16(B)
+    N, K = W.shape
+    rl = A.shape[1]
+    Wb = np.empty((N, K), dtype=np.uint16)
+    _load().oracle_lora_bake(_ptr(W), _ptr(A), _ptr(B), N, K, rl, float(scale), _ptr(Wb))
+    return Wb
+
+
+def quantize_sr(Y: np.ndarray, U: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row absmax INT4 scale, stochastic rounding with the given u."""
+    Y = np.ascontiguousarray(Y, dtype=np.float32)
+    U = np.ascontiguousarray(U, dtype=np.float32).reshape(Y.shape)
+    rows, K = Y.shape
+    q = np.empty((rows, K), dtype=np.int8)
+    s = np.empty((rows,), dtype=np.float32)
+    _load().oracle_quantize_sr(_ptr(Y), rows, K, _ptr(U), _ptr(q), _ptr(s))
+    return q, s
+
+
+def bake_requantize(W, A, B, scale: float, g: int, seed: int):
+    """LoRA baked into W, then rotated and stochastically rounded to INT4."""
+    Wb = lora_bake(W, A, B, scale)
+    Y = rotate(Wb, g)
+    q, s = quantize_sr(Y, sr_uniform(Y.size, seed).reshape(Y.shape))
+    return dict(w_baked=Wb, w_q=q, w_scale=s, w_packed=pack_int4(q))
 
 
 def gelu_tanh(x: np.ndarray) -> np.ndarray:

@@ -283,6 +283,92 @@ void oracle_lowrank_down(const uint16_t *X, const uint16_t *L1, long M, int K, i
         }
 }
 
+/* ---- baking a LoRA into the weights, stochastic-rounding re-quantization ---- */
+
+/* "ComfyUI-INT4-Fast" ("INT4 Quantized Inference Comes to ComfyUI") and the
+   toolkit page ("How the toolkit tells you to choose") let a LoRA be baked
+   into the 4-bit weights; re-quantizing W + dW rounds stochastically so the
+   small LoRA update survives 4-bit rounding in expectation.  Readings:
+     Wb[n][k] = bf16(fl32(W[n][k] + fl32(scale * sum_j A[k][j] B[j][n]))),
+   the sum as fp32 fused multiply-adds in index order j = 0, 1, ...;
+   codes after the usual rotation and absmax scale s = fl32(amax / 7):
+     q = clamp(floor(fl32(fl32(y / s) + u)), -8, 7),  u in [0, 1),
+   u drawn from Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
+   numbers: as easy as 1, 2, 3", SC 2011): element e of the row-major [N, K]
+   array takes word e % 4 of Philox(counter = (e / 4, 0, 0, 0),
+   key = (seed, 0)), and u = (word >> 40) * 2^-24 (24 random bits, exact in
+   fp32). */
+void oracle_philox4x64(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
+    const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+    uint64_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3], k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        const unsigned __int128 p0 = (unsigned __int128)M0 * c0;
+        const unsigned __int128 p1 = (unsigned __int128)M1 * c2;
+        const uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
+        const uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+        if (r < 9) {
+            k0 += W0;
+            k1 += W1;
+        }
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+void oracle_sr_uniform(long n, uint64_t seed, float *u) {
+    #pragma omp parallel for schedule(static)
+    for (long b = 0; b < (n + 3) / 4; ++b) {
+        const uint64_t ctr[4] = {(uint64_t)b, 0, 0, 0}, key[2] = {seed, 0};
+        uint64_t w[4];
+        oracle_philox4x64(ctr, key, w);
+        for (int l = 0; l < 4 && 4 * b + l < n; ++l) u[4 * b + l] = (float)(w[l] >> 40) * 0x1p-24f;
+    }
+}
+
+void oracle_lora_bake(const uint16_t *W, const uint16_t *A, const uint16_t *B, int N, int K, int rl, float scale,
+                      uint16_t *Wb) {
+    #pragma omp parallel for schedule(static)
+    for (long n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            float acc = 0.0f;
+            for (int j = 0; j < rl; ++j)
+                acc = fmaf(bf16_to_f32(A[(long)k * rl + j]), bf16_to_f32(B[(long)j * N + n]), acc);
+            const float d = scale * acc;
+            Wb[n * K + k] = f32_to_bf16(bf16_to_f32(W[n * K + k]) + d);
+        }
+}
+
+/* s = fl32(amax / 7) per row, q = clamp(floor(fl32(fl32(y / s) + u)), -8, 7);
+   a row with amax == 0 gets s = 0 and codes 0. */
+void oracle_quantize_sr(const float *Y, long rows, int K, const float *U, int8_t *q, float *scale) {
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        const float *y = Y + r * K;
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(y[k]);
+            if (a > amax) amax = a;
+        }
+        const float s = amax / 7.0f;
+        scale[r] = s;
+        for (int k = 0; k < K; ++k) {
+            int v = 0;
+            if (s != 0.0f) {
+                const float t = y[k] / s;
+                const float w = t + U[r * K + k];
+                v = (int)floorf(w);
+                if (v < -8) v = -8;
+                if (v > 7) v = 7;
+            }
+            q[r * K + k] = (int8_t)v;
+        }
+    }
+}
+
 /* GELU with the tanh approximation, in fp64 (the MLP between the up and down
    projections of the pages' diffusion transformer blocks, "Load Diffusion
    Model INT4 (W4A4)": every linear layer of the model runs in 4 bit, the

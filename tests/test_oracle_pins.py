@@ -24,6 +24,11 @@ textbook facts, library routines, closed forms and hand-derived fixtures):
     the layer is (X L1) L2 + s (X A) B + b in NumPy fp64, merged or not.
   * GELU(tanh): torch's tanh-approximate GELU in fp64; gelu(0) = 0,
     gelu(x) - gelu(-x) = x; the fused layer is GELU of the unrounded output.
+  * LoRA bake + stochastic rounding: Philox4x64-10 equals NumPy's Philox
+    bit generator; u layout and uniformity (chi-square, mean); codes are
+    floor or floor + 1 and unbiased over seeds; the bake is within one bf16
+    ulp (plus the fp32 sum bound) of W + s A B in fp64, and B = 0 is the
+    identity.
   * Planted mistakes (in copies of oracle outputs, on the CPU) are caught.
 """
 from __future__ import annotations
@@ -541,3 +546,80 @@ def test_gelu_layer_applies_after_the_epilogue():
     base = oracle.linear_w4a4(d["X"], d["W"], 64, d["L1"], d["L2"], d["bias"])
     assert np.array_equal(out["Y_linear"], base["Y"])
     assert np.array_equal(out["Y"], oracle.gelu_tanh(base["Y"]))
+
+
+# ---------------------------------------------------------------- LoRA bake + stochastic rounding
+@pytest.mark.parametrize("counter,key", [([0, 0, 0, 0], [0, 0]), ([5, 0, 0, 0], [0x1234, 0x99]),
+                                         ([2 ** 64 - 2, 7, 11, 13], [2 ** 63 + 5, 3]),
+                                         ([12345, 0, 0, 0], [0xDEADBEEF, 0])])
+def test_philox_matches_numpy(counter, key):
+    """Philox4x64-10 equals NumPy's Philox bit generator (which advances its
+    counter by one before producing the first block)."""
+    c = np.array(counter, dtype=np.uint64)
+    prev = c.copy()
+    # counter - 1 with borrow across the four words
+    for i in range(4):
+        if prev[i] != 0:
+            prev[i] -= np.uint64(1)
+            break
+        prev[i] = np.uint64(2 ** 64 - 1)
+    raw = np.random.Philox(counter=prev, key=np.array(key, dtype=np.uint64)).random_raw(4)
+    assert np.array_equal(oracle.philox4x64(c, np.array(key, dtype=np.uint64)), raw)
+
+
+def test_sr_uniform_layout_and_distribution():
+    """Element e takes word e % 4 of block e / 4 (top 24 bits), and the u are
+    uniform on [0, 1): chi-square over 64 bins, mean 1/2."""
+    n, seed = 1 << 18, 2024
+    u = oracle.sr_uniform(n, seed)
+    for e in (0, 1, 2, 3, 4, 4097, n - 1):
+        w = oracle.philox4x64(np.array([e // 4, 0, 0, 0], dtype=np.uint64), np.array([seed, 0], dtype=np.uint64))
+        assert u[e] == np.float32(int(w[e % 4]) >> 40) * np.float32(2.0 ** -24)
+    assert u.min() >= 0.0 and u.max() < 1.0
+    counts = np.bincount((u * 64).astype(np.int64), minlength=64)
+    chi2 = np.sum((counts - n / 64) ** 2 / (n / 64))
+    assert chi2 < 120.0                       # 63 degrees of freedom, p ~ 1e-5
+    assert abs(float(u.mean()) - 0.5) < 4.0 / np.sqrt(12 * n)
+    assert not np.array_equal(u[:64], oracle.sr_uniform(64, seed + 1))
+
+
+def test_sr_rounds_down_or_up_and_is_unbiased():
+    """Each code is floor(y/s) or that plus one (before the clamp); over many
+    seeds the mean code approaches y/s (unbiased rounding)."""
+    rng = np.random.default_rng(60)
+    Y = rng.standard_normal((4, 256)).astype(np.float32)
+    t = None
+    acc = np.zeros(Y.shape)
+    n_seeds = 400
+    for seed in range(n_seeds):
+        q, s = oracle.quantize_sr(Y, oracle.sr_uniform(Y.size, seed).reshape(Y.shape))
+        t = Y.astype(np.float64) / s.astype(np.float64)[:, None]
+        fl = np.floor(t)
+        assert np.all((q == fl) | (q == fl + 1) | (q == 7) | (q == -8))
+        acc += q
+    mean = acc / n_seeds
+    # standard error of a Bernoulli mean <= 0.5 / sqrt(n)
+    assert np.max(np.abs(mean - t)) < 5 * 0.5 / np.sqrt(n_seeds)
+    # planted mistake: deterministic rounding is biased on this data
+    q_rn, _ = oracle.quantize(Y, 7)
+    assert np.max(np.abs(q_rn - t)) > 0.4
+
+
+def test_lora_bake_bound_and_identities():
+    """Wb within one bf16 ulp (plus the fp32 sum error) of W + s A B in fp64;
+    B = 0 leaves W unchanged; the baked layer's weights feed the usual
+    rotation."""
+    rng = np.random.default_rng(61)
+    N, K, rl = 48, 256, 32
+    W = _bf16(rng.standard_normal((N, K), dtype=np.float32) * 0.02)
+    A = _bf16(rng.standard_normal((K, rl), dtype=np.float32) * 0.1)
+    B = _bf16(rng.standard_normal((rl, N), dtype=np.float32) * 0.1)
+    Wb = oracle.lora_bake(W, A, B, 0.75)
+    f = oracle.bf16_to_f64
+    exact = f(W) + 0.75 * (f(A) @ f(B)).T
+    sum_err = 0.75 * rl * 2.0 ** -23 * (np.abs(f(A)) @ np.abs(f(B))).T
+    assert np.all(np.abs(f(Wb) - exact) <= 2.0 ** -8 * np.abs(exact) + 2 * sum_err + 1e-30)
+    assert np.array_equal(oracle.lora_bake(W, A, np.zeros_like(B), 0.75), W)
+    out = oracle.bake_requantize(W, A, B, 0.75, 64, seed=9)
+    assert np.array_equal(out["w_baked"], Wb)
+    assert np.all(np.abs(out["w_q"]) <= 8)
