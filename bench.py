@@ -297,6 +297,49 @@ def run_mlp(args):
     print(json.dumps(line), flush=True)
 
 
+def run_bake(args):
+    """Baking a LoRA of rank --bake-lora into the attention-projection weights
+    (N = K = 3072, g = 128) and re-quantizing them with stochastic rounding:
+    the fp32 bake kernel and the stochastic-rounding rotate + quantize, per
+    call.  An offline step (once per LoRA change), reported as time."""
+    import torch
+    import w4a4_int4_quantized_b200 as w4
+    from w4a4_int4_quantized_b200 import inputs
+    w4.load_library()
+    spec = inputs.WORKLOADS["attn_proj"]
+    N, K, g, rl = spec.N, spec.K, spec.group, args.bake_lora
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    W = dev(inputs.make_layer(spec)["W"])
+    A = dev(inputs.random_bf16((K, rl), seed=11, std=0.05))
+    B = dev(inputs.random_bf16((rl, N), seed=12, std=0.05))
+    Wb = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    Wq = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    ws = torch.empty((N,), dtype=torch.float32, device="cuda")
+    for i in range(args.warmup):
+        w4.w4a4_bake_lora_sr(W, A, B, 1.0, g, i, W_baked=Wb, Wq=Wq, w_scale=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        w4.w4a4_bake_lora_sr(W, A, B, 1.0, g, 1000 + i, W_baked=Wb, Wq=Wq, w_scale=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / args.steps * 1e3
+    err = w4.w4a4_get_device_error()
+    if err:
+        raise SystemExit(f"device error word {err:#x}")
+    print(json.dumps({
+        "metric": f"LoRA bake (rank {rl}) + stochastic-rounding INT4 re-quantization, us per call (N=K=3072)",
+        "value": us, "unit": "us", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 bake, int4 out",
+        "data": "synthetic", "config": {"workload": "attn_proj_weights_bake", "N": N, "K": K, "group": g,
+                                        "lora_rank": rl},
+        "gpu_launches": 2 * args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -307,6 +350,8 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--bake-lora", type=int, default=0,
+                    help="time baking a LoRA of this rank into the weights with stochastic re-quantization")
     ap.add_argument("--mlp", action="store_true",
                     help="time the fused MLP pair (up with GELU in its epilogue, then down) instead")
     ap.add_argument("--lora", type=int, default=0,
@@ -318,6 +363,12 @@ def main():
         raise SystemExit("--warmup must be >= 3")
 
     from w4a4_int4_quantized_b200 import inputs
+    if args.bake_lora:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the bake is measured by the GPU arm only"}))
+            return
+        run_bake(args)
+        return
     if args.mlp:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the MLP chain is measured by the GPU arm only"}))

@@ -259,6 +259,27 @@ w4a4_status w4a4_mlp(const void* X, int M, int D, int H, int group, const uint8_
 w4a4_status w4a4_lora_merge(const void* L1, const void* L2, int rank, const void* A, const void* B, int lora_rank,
                             float lora_scale, int K, int N, void* L1_out, void* L2_out, w4a4_stream_t stream);
 
+/* ---------------------------------------------------------------- LoRA baking */
+/* Bakes a LoRA into the weights and re-quantizes them with stochastic
+ * rounding ("ComfyUI-INT4-Fast", "INT4 Quantized Inference Comes to
+ * ComfyUI", and "W4A4 and W4A8: The New Quantization Toolkit", "How the
+ * toolkit tells you to choose": a LoRA can be merged into the 4-bit
+ * weights; rounding stochastically keeps the small update in expectation).
+ *   W_baked [N, K] = bf16(fl32(W + fl32(lora_scale * sum_j A[k][j] B[j][n])))
+ * (fp32 fused multiply-adds over j in index order), then the W4A4 weight
+ * routine (rotation, s = fl32(amax / 7) per row) with
+ *   q = clamp(floor(fl32(fl32(y / s) + u)), -8, 7),
+ * u in [0, 1) from Philox4x64-10 (Salmon et al., SC 2011): element e of the
+ * row-major [N, K] codes uses word e % 4 of Philox(counter = (e / 4, 0, 0, 0),
+ * key = (seed, 0)), top 24 bits times 2^-24.  W [N, K], A [K, lora_rank],
+ * B [lora_rank, N]: bf16; W_baked (output, [N, K] bf16), Wq [N, K/2] and
+ * w_scale [N] as w4a4_quantize_weights; 16-byte aligned device memory.
+ * 1 <= lora_rank <= 256; K and group as w4a4_quantize_weights.  The result
+ * is deterministic for a given seed. */
+w4a4_status w4a4_bake_lora_sr(const void* W, const void* A, const void* B, int lora_rank, float lora_scale, int N,
+                              int K, int group, unsigned long long seed, void* W_baked, uint8_t* Wq, float* w_scale,
+                              w4a4_stream_t stream);
+
 /* ---------------------------------------------------------------- failures */
 /* Kernels never trap: a wait on another part of the kernel that runs past its
  * time limit (2 s) records a code in a per-device error word and lets the

@@ -47,7 +47,7 @@ def test_header_declares_the_documented_entry_points():
               "w4a4_workspace_bytes", "w8a8_workspace_bytes", "w4a4_status_string", "w4a4_version",
               "w4a4_get_device_error", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear",
               "w4a8_workspace_bytes", "w4a4_lora_merge", "w4a4_gemm_gelu", "w4a4_linear_gelu", "w4a4_mlp",
-              "w4a4_mlp_workspace_bytes"]:
+              "w4a4_mlp_workspace_bytes", "w4a4_bake_lora_sr"]:
         assert n in names
 
 
@@ -129,6 +129,19 @@ def test_mlp_workspace_and_validation(lib):
     g = lib.w4a4_gemm_gelu
     assert g(A, B, C, D, 64, 12, 256, 64, NUL, NUL, 0, NUL, E, NUL, NUL) == SHAPE
     assert lib.w4a4_linear_gelu(A, B, C, 64, 256, 256, 64, NUL, NUL, 0, NUL, D, E, 1, NUL) == WORKSPACE
+
+
+def test_bake_lora_sr_validation(lib):
+    f = lib.w4a4_bake_lora_sr
+    args = [A, B, C, 16, 0.5, 64, 256, 128, 7, D, E, E, NUL]
+    bad = list(args); bad[2] = NUL
+    assert f(*bad) == INVALID
+    bad = list(args); bad[3] = 0                      # no LoRA rank
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[6] = 320                    # K not a multiple of 128
+    assert f(*bad) == SHAPE
+    bad = list(args); bad[9] = ODD
+    assert f(*bad) == MISALIGNED
 
 
 def test_lora_merge_validation(lib):

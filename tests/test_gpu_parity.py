@@ -316,6 +316,28 @@ def test_fused_mlp_chain():
     check_output(host_f64(Y), ref_y["Y"], lowrank=True)
 
 
+@pytest.mark.parametrize("N,K,g,rl,scale,seed", [(264, 640, 64, 16, 0.5, 1), (96, 3072, 128, 64, 1.3, 77),
+                                                 (40, 12288, 128, 32, 0.7, 2 ** 63 + 11), (64, 256, 0, 16, 2.0, 5)])
+def test_bake_lora_sr_bitexact(N, K, g, rl, scale, seed):
+    """LoRA baked into W (bf16, fp32 index-order FMA sums) and stochastically
+    re-quantized with Philox4x64-10: the baked weights, scales and codes are
+    bit-identical to the oracle's, and a second call with the same seed
+    repeats them."""
+    import torch
+    W = inputs.random_bf16((N, K), seed=N + K, std=0.02)
+    A = inputs.random_bf16((K, rl), seed=rl, std=0.05)
+    B = inputs.random_bf16((rl, N), seed=rl + 1, std=0.05)
+    Wb, Wq, ws = w4.w4a4_bake_lora_sr(dev_bf16(W), dev_bf16(A), dev_bf16(B), scale, g, seed)
+    torch.cuda.synchronize()
+    ref = oracle.bake_requantize(W, A, B, scale, g, seed)
+    assert np.array_equal(Wb.cpu().view(torch.int16).numpy().view(np.uint16), ref["w_baked"])
+    assert np.array_equal(ws.cpu().numpy().view(np.uint32), ref["w_scale"].view(np.uint32))
+    got = Wq.cpu().numpy()
+    assert np.array_equal(got, ref["w_packed"]), f"{np.count_nonzero(got != ref['w_packed'])} code bytes differ"
+    _, Wq2, _ = w4.w4a4_bake_lora_sr(dev_bf16(W), dev_bf16(A), dev_bf16(B), scale, g, seed)
+    assert torch.equal(Wq2, Wq)
+
+
 def test_attn_proj_full_size_sampled():
     """The attention-projection workload at full size (M=4608, K=N=3072,
     g=128, bias), in the launch configuration the benchmark times

@@ -23,7 +23,7 @@ __all__ = [
     "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
     "w8a8_workspace_bytes", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear", "w4a8_workspace_bytes",
     "w4a4_lora_merge", "w4a4_gemm_gelu", "w4a4_linear_gelu", "w4a4_mlp", "w4a4_mlp_workspace_bytes",
-    "w4a4_get_device_error",
+    "w4a4_bake_lora_sr", "w4a4_get_device_error",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -79,6 +79,7 @@ def load_library():
         "w4a4_gemm_gelu": ([P, P, P, P, I, I, I, I, P, P, I, P, P, P, P], S),
         "w4a4_linear_gelu": ([P, P, P, I, I, I, I, P, P, I, P, P, P, Z, P], S),
         "w4a4_mlp_workspace_bytes": ([I, I, I, I, I], Z),
+        "w4a4_bake_lora_sr": ([P, P, P, I, ctypes.c_float, I, I, I, ctypes.c_ulonglong, P, P, P, P], S),
         "w4a4_mlp": ([P, I, I, I, I, P, P, P, P, I, P, P, P, P, P, I, P, P, P, Z, P], S),
         "w4a4_get_device_error": ([P, ctypes.POINTER(ctypes.c_uint)], S),
     }
@@ -353,6 +354,22 @@ def w4a4_mlp(X, group, up, down, Y=None, workspace=None, stream=None):
         _ptr(down.get("L2")), rd, _ptr(down.get("bias")), _ptr(Y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return Y
+
+
+def w4a4_bake_lora_sr(W, A, B, lora_scale: float, group: int, seed: int, W_baked=None, Wq=None, w_scale=None,
+                      stream=None):
+    """LoRA baked into W, then rotated and stochastically rounded to INT4:
+    (W_baked bf16 [N, K], packed codes [N, K/2], scales [N])."""
+    import torch
+    N, K = W.shape
+    rl = A.shape[1]
+    W_baked = _empty((N, K), torch.bfloat16, W) if W_baked is None else W_baked
+    Wq = _empty((N, K // 2), torch.uint8, W) if Wq is None else Wq
+    w_scale = _empty((N,), torch.float32, W) if w_scale is None else w_scale
+    _check("w4a4_bake_lora_sr", load_library().w4a4_bake_lora_sr(
+        _ptr(W), _ptr(A), _ptr(B), rl, float(lora_scale), N, K, group, int(seed), _ptr(W_baked), _ptr(Wq),
+        _ptr(w_scale), _stream(stream)))
+    return W_baked, Wq, w_scale
 
 
 def w4a4_get_device_error(stream=None) -> int:

@@ -354,6 +354,26 @@ w4a4_status w4a4_lora_merge(const void* L1, const void* L2, int rank, const void
                                        static_cast<uint16_t*>(L2_out), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+w4a4_status w4a4_bake_lora_sr(const void* W, const void* A, const void* B, int lora_rank, float lora_scale, int N,
+                              int K, int group, unsigned long long seed, void* W_baked, uint8_t* Wq, float* w_scale,
+                              w4a4_stream_t stream) {
+  if (!W || !A || !B || !W_baked || !Wq || !w_scale) return W4A4_ERR_INVALID_ARG;
+  if (lora_rank < 1 || lora_rank > 256 || N < 1) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  w4a4_status s = check_k_group(K, group);
+  if (s != W4A4_OK) return s;
+  if (!aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(W_baked) || !aligned16(Wq) ||
+      !aligned16(w_scale))
+    return W4A4_ERR_MISALIGNED;
+  if ((s = check_device()) != W4A4_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_lora_bake(static_cast<const uint16_t*>(W), static_cast<const uint16_t*>(A),
+                                   static_cast<const uint16_t*>(B), N, K, lora_rank, lora_scale,
+                                   static_cast<uint16_t*>(W_baked), st);
+  if (e != cudaSuccess) return W4A4_ERR_CUDA;
+  return cuda_status(launch_rotate_quantize_sr(static_cast<const uint16_t*>(W_baked), N, K, group, Wq, w_scale,
+                                               seed, st));
+}
+
 // ------------------------------------------------------------------ failures
 w4a4_status w4a4_get_device_error(w4a4_stream_t stream, unsigned int* code) {
   w4a4_status s = check_device();

@@ -38,6 +38,15 @@ cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st);
 cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
                                 cudaStream_t st);
 
+// Symmetric INT4 codes of rotated rows with stochastic rounding: q =
+// clamp(floor(y / s + u), -8, 7), u from Philox4x64-10 keyed by `seed`.
+cudaError_t launch_rotate_quantize_sr(const uint16_t* X, int rows, int K, int group, uint8_t* out, float* scale,
+                                      unsigned long long seed, cudaStream_t st);
+
+// Wb [N, K] = bf16(W + scale * (A B)^T), fp32 FMA sums in index order.
+cudaError_t launch_lora_bake(const uint16_t* W, const uint16_t* A, const uint16_t* B, int N, int K, int rl,
+                             float scale, uint16_t* Wb, cudaStream_t st);
+
 // [L1 | A] and [L2 ; bf16(fl32(scale * B))] (rank r + rl low-rank operands).
 cudaError_t launch_lora_merge(const uint16_t* L1, const uint16_t* L2, int r, const uint16_t* A, const uint16_t* B,
                               int rl, float scale, int K, int N, uint16_t* L1o, uint16_t* L2o, cudaStream_t st);

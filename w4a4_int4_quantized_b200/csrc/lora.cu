@@ -58,7 +58,36 @@ __global__ void lora_merge_kernel(const uint16_t* __restrict__ L1, const uint16_
   }
 }
 
+// Wb[n][k] = bf16(fl32(W[n][k] + fl32(scale * sum_j A[k][j] B[j][n]))), the
+// sum as fp32 fused multiply-adds in index order (the reading of baking a
+// LoRA into the weights before they are re-quantized).  One thread per
+// output; a warp covers consecutive k of one weight row n, so B[j][n] is a
+// broadcast and A's rows are read in order.
+__global__ void lora_bake_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__ A,
+                                 const uint16_t* __restrict__ B, int N, int K, int rl, float scale,
+                                 uint16_t* __restrict__ Wb) {
+  const int n = blockIdx.y;
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N || k >= K) return;
+  float acc = 0.0f;
+  for (int j = 0; j < rl; ++j) {
+    const float a = __uint_as_float((uint32_t)A[(long)k * rl + j] << 16);
+    const float b = __uint_as_float((uint32_t)B[(long)j * N + n] << 16);
+    acc = __fmaf_rn(a, b, acc);
+  }
+  const float w = __uint_as_float((uint32_t)W[(long)n * K + k] << 16);
+  const __nv_bfloat16 h = __float2bfloat16_rn(__fadd_rn(w, __fmul_rn(scale, acc)));
+  Wb[(long)n * K + k] = *reinterpret_cast<const uint16_t*>(&h);
+}
+
 }  // namespace
+
+cudaError_t launch_lora_bake(const uint16_t* W, const uint16_t* A, const uint16_t* B, int N, int K, int rl,
+                             float scale, uint16_t* Wb, cudaStream_t st) {
+  const dim3 grid((unsigned)((K + 255) / 256), (unsigned)N);
+  lora_bake_kernel<<<grid, 256, 0, st>>>(W, A, B, N, K, rl, scale, Wb);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_lora_merge(const uint16_t* L1, const uint16_t* L2, int r, const uint16_t* A, const uint16_t* B,
                               int rl, float scale, int K, int N, uint16_t* L1o, uint16_t* L2o, cudaStream_t st) {

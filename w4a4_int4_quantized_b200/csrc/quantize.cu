@@ -117,6 +117,61 @@ __device__ __forceinline__ void quantize_block8(const float2* P8, float2 ih, flo
 // registers held while in flight), so the loads of the next blocks overlap
 // the rotation and quantization of the current one.  One thread owns one
 // group; its g values go from shared memory straight into float2 registers.
+// Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011): 10 rounds of two 64 x 64 -> 128-bit products
+// on a 4-word counter with a Weyl-sequence key schedule.
+__device__ __forceinline__ void philox4x64_10(uint64_t c[4], uint64_t k0, uint64_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t m0 = 0xD2E7470EE14C6C93ull, m1 = 0xCA5A826395121157ull;
+    const uint64_t hi0 = __umul64hi(m0, c[0]), lo0 = m0 * c[0];
+    const uint64_t hi1 = __umul64hi(m1, c[2]), lo1 = m1 * c[2];
+    const uint64_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+    k0 += 0x9E3779B97F4A7C15ull;
+    k1 += 0xBB67AE8584CAA73Bull;
+  }
+}
+
+// u in [0, 1) of elements e0 .. e0 + 7 (e0 a multiple of 4): element e takes
+// word e % 4 of Philox(counter = (e / 4, 0, 0, 0), key = (seed, 0)), top 24 bits.
+__device__ __forceinline__ void sr_uniform8(uint64_t e0, uint64_t seed, float (&u)[8]) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    uint64_t c[4] = {(e0 >> 2) + (uint64_t)b, 0ull, 0ull, 0ull};
+    philox4x64_10(c, seed, 0ull);
+#pragma unroll
+    for (int l = 0; l < 4; ++l) u[4 * b + l] = (float)(uint32_t)(c[l] >> 40) * 0x1p-24f;
+  }
+}
+
+// Stochastic rounding of 16 elements (8 float2 pairs; .x lanes are elements
+// ex0 .. ex0 + 7, .y lanes ey0 .. ey0 + 7 of the row-major array) to INT4
+// codes q = clamp(floor(fl32(fl32(y / s) + u)), -8, 7), packed as in the
+// round-to-nearest form.
+__device__ __forceinline__ void quantize_block8_sr(const float2* P8, float s, uint64_t ex0, uint64_t ey0,
+                                                   uint64_t seed, uint32_t* bw) {
+  float ux[8], uy[8];
+  sr_uniform8(ex0, seed, ux);
+  sr_uniform8(ey0, seed, uy);
+  uint32_t tx[8], ty[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    int qx = 0, qy = 0;
+    if (s != 0.0f) {
+      qx = min(max(__float2int_rd(__fadd_rn(__fdiv_rn(P8[j].x, s), ux[j])), -8), 7);
+      qy = min(max(__float2int_rd(__fadd_rn(__fdiv_rn(P8[j].y, s), uy[j])), -8), 7);
+    }
+    tx[j] = (uint32_t)qx;   // pack_nibbles8 keeps the low nibble
+    ty[j] = (uint32_t)qy;
+  }
+  bw[0] = pack_nibbles8(tx);
+  bw[1] = pack_nibbles8(ty);
+}
+
 // Order-preserving unsigned key of a float (for shared-memory atomic min/max).
 __device__ __forceinline__ uint32_t fkey(float v) {
   const uint32_t b = __float_as_uint(v);
@@ -130,10 +185,12 @@ __device__ __forceinline__ float fkey_value(uint32_t k) {
 // 4-bit with a zero point (W4A8 weights, packed unsigned codes): per row
 // s = fl32(fl32(max - min) / 15), z = clamp(rint(fl32(-min / s)), 0, 15),
 // q = clamp(rint(fl32(y / s)) + z, 0, 15), zero point written to `zero`.
-template <int G, bool ROT, int QMAX, int MAXT>
+// SR (QMAX 7 only): stochastic rounding with Philox4x64-10 under `seed`
+// instead of round-to-nearest (re-quantizing weights with a baked LoRA).
+template <int G, bool ROT, int QMAX, int MAXT, bool SR = false>
 __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
     rotate_quantize_kernel(const uint16_t* __restrict__ X, int M, int K, int rows_per_blk, uint8_t* __restrict__ out,
-                           float* __restrict__ scale, uint8_t* __restrict__ zero) {
+                           float* __restrict__ scale, uint8_t* __restrict__ zero, unsigned long long seed) {
   constexpr int HALF = G / 2;
   constexpr bool ASYM = (QMAX == 15);
   constexpr bool INT4 = (QMAX == 7) || ASYM;
@@ -297,9 +354,14 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
       for (int b = 0; b < SB; ++b) {
         const int blk8 = c * SB + b;
         uint32_t bw[INT4 ? 2 : 4];
-        uint32_t bad = 0u;
-        quantize_block8<INT4, false, ASYM>(P + 8 * blk8, ih, il, s, bw, bad, zoff);
-        if (bad) quantize_block8<INT4, true, ASYM>(P + 8 * blk8, ih, il, s, bw, bad, zoff);
+        if constexpr (SR) {
+          const uint64_t e0 = (uint64_t)row * (uint64_t)K + (uint64_t)(grp * G + 8 * blk8);
+          quantize_block8_sr(P + 8 * blk8, s, e0, e0 + HALF, seed, bw);
+        } else {
+          uint32_t bad = 0u;
+          quantize_block8<INT4, false, ASYM>(P + 8 * blk8, ih, il, s, bw, bad, zoff);
+          if (bad) quantize_block8<INT4, true, ASYM>(P + 8 * blk8, ih, il, s, bw, bad, zoff);
+        }
         if (INT4) {
           w[b] = bw[0];
           w[SB + b] = bw[1];
@@ -328,9 +390,9 @@ struct RqShape {
   int rows_per_blk, threads, smem, grid;
 };
 
-template <int G, bool ROT, int QMAX, int MAXT>
+template <int G, bool ROT, int QMAX, int MAXT, bool SR>
 cudaError_t pick_shape(int M, int K, int dev, RqShape& out) {
-  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT>;
+  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT, SR>;
   const int gpr = K / G;
   const int max_r = gpr >= MAXT ? 1 : MAXT / gpr;
   int sms = 148;
@@ -358,10 +420,10 @@ cudaError_t pick_shape(int M, int K, int dev, RqShape& out) {
   return cudaSuccess;
 }
 
-template <int G, bool ROT, int QMAX, int MAXT>
+template <int G, bool ROT, int QMAX, int MAXT, bool SR = false>
 cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* scale, uint8_t* zero,
-                        cudaStream_t st) {
-  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT>;
+                        unsigned long long seed, cudaStream_t st) {
+  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT, SR>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -380,7 +442,7 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
   if (dev < 64 && cache_m[dev] == M && cache_k[dev] == K) {
     sh = cache_shape[dev];
   } else {
-    if ((e = pick_shape<G, ROT, QMAX, MAXT>(M, K, dev, sh)) != cudaSuccess) return e;
+    if ((e = pick_shape<G, ROT, QMAX, MAXT, SR>(M, K, dev, sh)) != cudaSuccess) return e;
     if (dev < 64) {
       cache_shape[dev] = sh;
       cache_m[dev] = M;
@@ -397,25 +459,26 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, sh.rows_per_blk, out, scale, zero);
+  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, sh.rows_per_blk, out, scale, zero, seed);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 // Rows of up to 128 groups run in 128-thread CTAs (three per SM); wider rows
 // (K / g > 128) in 256-thread CTAs, one group per thread either way.
-template <int G, bool ROT, int QMAX>
-cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scale, uint8_t* zero, cudaStream_t st) {
-  if (K / G <= 128) return launch_rq_t<G, ROT, QMAX, 128>(X, M, K, out, scale, zero, st);
-  return launch_rq_t<G, ROT, QMAX, 256>(X, M, K, out, scale, zero, st);
+template <int G, bool ROT, int QMAX, bool SR = false>
+cudaError_t launch_rq(const uint16_t* X, int M, int K, uint8_t* out, float* scale, uint8_t* zero,
+                      unsigned long long seed, cudaStream_t st) {
+  if (K / G <= 128) return launch_rq_t<G, ROT, QMAX, 128, SR>(X, M, K, out, scale, zero, seed, st);
+  return launch_rq_t<G, ROT, QMAX, 256, SR>(X, M, K, out, scale, zero, seed, st);
 }
 
-template <int QMAX>
+template <int QMAX, bool SR = false>
 cudaError_t launch_rq_group(const uint16_t* X, int rows, int K, int group, uint8_t* out, float* scale, uint8_t* zero,
-                            cudaStream_t st) {
-  if (group == 64) return launch_rq<64, true, QMAX>(X, rows, K, out, scale, zero, st);
-  if (group == 128) return launch_rq<128, true, QMAX>(X, rows, K, out, scale, zero, st);
-  return launch_rq<128, false, QMAX>(X, rows, K, out, scale, zero, st);
+                            unsigned long long seed, cudaStream_t st) {
+  if (group == 64) return launch_rq<64, true, QMAX, SR>(X, rows, K, out, scale, zero, seed, st);
+  if (group == 128) return launch_rq<128, true, QMAX, SR>(X, rows, K, out, scale, zero, seed, st);
+  return launch_rq<128, false, QMAX, SR>(X, rows, K, out, scale, zero, seed, st);
 }
 
 }  // namespace
@@ -426,9 +489,15 @@ cudaError_t launch_rq_group(const uint16_t* X, int rows, int K, int group, uint8
 // group 0 turns the rotation off.  Shapes are validated by the caller.
 cudaError_t launch_rotate_quantize(const uint16_t* X, int rows, int K, int group, int qmax, uint8_t* out,
                                    float* scale, uint8_t* zero, cudaStream_t st) {
-  if (qmax == 7) return launch_rq_group<7>(X, rows, K, group, out, scale, nullptr, st);
-  if (qmax == 15) return launch_rq_group<15>(X, rows, K, group, out, scale, zero, st);
-  return launch_rq_group<127>(X, rows, K, group, out, scale, nullptr, st);
+  if (qmax == 7) return launch_rq_group<7>(X, rows, K, group, out, scale, nullptr, 0ull, st);
+  if (qmax == 15) return launch_rq_group<15>(X, rows, K, group, out, scale, zero, 0ull, st);
+  return launch_rq_group<127>(X, rows, K, group, out, scale, nullptr, 0ull, st);
+}
+
+// Symmetric INT4 with stochastic rounding (Philox4x64-10 under `seed`).
+cudaError_t launch_rotate_quantize_sr(const uint16_t* X, int rows, int K, int group, uint8_t* out, float* scale,
+                                      unsigned long long seed, cudaStream_t st) {
+  return launch_rq_group<7, true>(X, rows, K, group, out, scale, nullptr, seed, st);
 }
 
 }  // namespace w4a4
