@@ -42,9 +42,9 @@ HBM_NOMINAL_GBS = 8000.0
 # they were taken from (sha256 prefix); reported as null once the source
 # changes.
 MEASURED_TRAFFIC = {
-    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "5a6b710f1ec7a816", 11.880448e6 + 0.05504e6),
-    "gemm_w4a8": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "5a6b710f1ec7a816", 18.96192e6 + 0.114176e6),
-    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "0a39f00184b08d94", 28.377856e6),
+    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "e37d2d655d741551", 11.880192e6 + 0.041472e6),
+    "gemm_w4a8": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "e37d2d655d741551", 18.961664e6 + 0.24448e6),
+    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "61d3e84e299a0ca7", 28.377344e6),
 }
 
 
@@ -289,9 +289,9 @@ def run_mlp(args):
         "dtype": "int4 codes (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
         "config": {"workload": "mlp_pair", "M": M, "D": D, "H": H, "group": g, "rank": r,
                    "l2": "2 rotating input sets; [M, 12288] intermediates exceed L2"},
-        "roofline": {"bound": "tensor", "achieved": ops / (ms * 1e-3) / 1e12, "peak": 2.0 * pk["bf16_sustained"],
-                     "unit": "TOPS", "frac": ops / (ms * 1e-3) / 1e12 / (2.0 * pk["bf16_sustained"]),
-                     "traffic": None, "peak_note": "whole chain against the int8 tensor peak"},
+        "roofline": {"bound": "tensor", "achieved": ops / (ms * 1e-3) / 1e12, "peak": 2.0 * pk["bf16"],
+                     "unit": "TOPS", "frac": ops / (ms * 1e-3) / 1e12 / (2.0 * pk["bf16"]),
+                     "traffic": None, "peak_note": "whole chain against the int8 tensor peak (2 x burst bf16)"},
         "gpu_launches": 6 * args.steps, "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -533,7 +533,9 @@ def main():
         k1 = k1_ms
         k2 = k2_ms
         k2_tops = ops / (k2 * 1e-3) / 1e12
-        int8_peak = 2.0 * pk["bf16_sustained"]   # nominal int8 : bf16 ratio is 2
+        # the GEMM is timed alone in a short back-to-back loop at full clock:
+        # the burst bf16 figure x the nominal int8 : bf16 ratio of 2
+        int8_peak = 2.0 * pk["bf16"]
         k1_bytes = M * K * 2 + (M * K if w4a8 else M * K // 2) + M * 4
         line = {
             "metric": _metric_name(args.variant, spec),
@@ -551,7 +553,8 @@ def main():
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
                          "frac": k2_tops / int8_peak,
                          "traffic": _traffic("gemm_w4a8" if w4a8 else "gemm", spec.name),
-                         "peak_note": f"int8 = 2 x {pk['source']} sustained bf16 {pk['bf16_sustained']} TFLOP/s"},
+                         "peak_note": f"int8 = 2 x {pk['source']} burst bf16 {pk['bf16']} TFLOP/s (kernel timed "
+                                      f"alone); {2.0 * pk['bf16_sustained']:.0f} with the sustained figure"},
             "roofline_k1": {"bound": "hbm", "achieved": k1_bytes / (k1 * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": k1_bytes / (k1 * 1e-3) / 1e9 / pk["hbm_gbs"],
                             "traffic": None if w4a8 else _traffic("rotate_quantize", spec.name)},
