@@ -366,5 +366,39 @@ def test_attn_proj_full_size_sampled():
     check_output(host_f64(Y)[rows], y_ref, lowrank=False)
 
 
+@pytest.mark.parametrize("name", ["mlp_up", "mlp_down"])
+def test_mlp_layers_full_size_sampled(name):
+    """The MLP layers at full size (M=4608, 3072->12288 and 12288->3072,
+    g=128, r=128, bias) in the benchmark's launch configuration
+    (w4a4_linear), on sampled token rows: weight and activation codes and
+    scales, the low-rank T, bit-exact accumulators of those rows, outputs
+    within the low-rank tolerance."""
+    import torch
+    spec = inputs.WORKLOADS[name]
+    d = inputs.make_layer(spec)
+    X, W, b = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    L1, L2 = dev_bf16(d["L1"]), dev_bf16(d["L2"])
+    Wq, ws = w4.w4a4_quantize_weights(W, spec.group)
+    Y = w4.w4a4_linear(X, Wq, ws, spec.group, L1, L2, b)
+    Xq, xs, T = w4.w4a4_rotate_quantize_act(X, spec.group, L1)
+    acc = torch.empty((spec.M, spec.N), dtype=torch.int32, device="cuda")
+    w4.w4a4_gemm(Xq, xs, Wq, ws, spec.group, T, L2, b, acc_debug=acc)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(6).choice(spec.M, size=24, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, spec.M - 1]]))
+    wp, wsr, wq = oracle.quantize_w4(d["W"], spec.group)
+    assert np.array_equal(Wq.cpu().numpy(), wp)
+    assert np.array_equal(ws.cpu().numpy(), wsr)
+    xp, xsr, xq = oracle.quantize_w4(d["X"][rows], spec.group)
+    assert np.array_equal(Xq.cpu().numpy()[rows], xp)
+    assert np.array_equal(xs.cpu().numpy()[rows], xsr)
+    acc_ref = oracle.int_gemm(xq, wq)
+    assert np.array_equal(acc.cpu().numpy()[rows], acc_ref)
+    t_ref = oracle.lowrank_down(d["X"][rows], d["L1"])
+    assert np.max(np.abs(host_f64(T)[rows] - t_ref)) <= 1e-2 * np.max(np.abs(t_ref))
+    y_ref = oracle.epilogue(acc_ref, xsr, wsr, spec.group, t_ref, d["L2"], d["bias"])
+    check_output(host_f64(Y)[rows], y_ref, lowrank=True)
+
+
 def test_no_device_error_after_runs():
     assert w4.w4a4_get_device_error() == 0
