@@ -60,31 +60,68 @@ __global__ void lora_merge_kernel(const uint16_t* __restrict__ L1, const uint16_
 
 // Wb[n][k] = bf16(fl32(W[n][k] + fl32(scale * sum_j A[k][j] B[j][n]))), the
 // sum as fp32 fused multiply-adds in index order (the reading of baking a
-// LoRA into the weights before they are re-quantized).  One thread per
-// output; a warp covers consecutive k of one weight row n, so B[j][n] is a
-// broadcast and A's rows are read in order.
-__global__ void lora_bake_kernel(const uint16_t* __restrict__ W, const uint16_t* __restrict__ A,
-                                 const uint16_t* __restrict__ B, int N, int K, int rl, float scale,
-                                 uint16_t* __restrict__ Wb) {
-  const int n = blockIdx.y;
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N || k >= K) return;
-  float acc = 0.0f;
-  for (int j = 0; j < rl; ++j) {
-    const float a = __uint_as_float((uint32_t)A[(long)k * rl + j] << 16);
-    const float b = __uint_as_float((uint32_t)B[(long)j * N + n] << 16);
-    acc = __fmaf_rn(a, b, acc);
+// LoRA into the weights before they are re-quantized).  A CTA computes a
+// 64 (n) x 64 (k) tile; A and B are staged through shared memory in chunks
+// of 32 ranks taken in order, so every output's FMA chain still runs
+// j = 0, 1, 2, ... and the result is bit-exact.  Each thread owns 4 x 4
+// outputs (k fastest, for coalesced stores).
+constexpr int kBakeTile = 64;
+constexpr int kBakeChunk = 32;
+
+__global__ void __launch_bounds__(256) lora_bake_kernel(const uint16_t* __restrict__ W,
+                                                        const uint16_t* __restrict__ A,
+                                                        const uint16_t* __restrict__ B, int N, int K, int rl,
+                                                        float scale, uint16_t* __restrict__ Wb) {
+  __shared__ float As[kBakeChunk][kBakeTile + 1];   // [j][k]
+  __shared__ float Bs[kBakeChunk][kBakeTile + 1];   // [j][n]
+  const int k0 = blockIdx.x * kBakeTile, n0 = blockIdx.y * kBakeTile;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int j0 = 0; j0 < rl; j0 += kBakeChunk) {
+    for (int t = threadIdx.x; t < kBakeChunk * kBakeTile; t += blockDim.x) {
+      const int jj = t % kBakeChunk, kk = t / kBakeChunk;          // A[k][j]: j fastest in memory
+      const int k = k0 + kk, j = j0 + jj;
+      As[jj][kk] = (k < K && j < rl) ? __uint_as_float((uint32_t)A[(long)k * rl + j] << 16) : 0.0f;
+      const int nn = t % kBakeTile, jb = t / kBakeTile;            // B[j][n]: n fastest in memory
+      const int n = n0 + nn, j2 = j0 + jb;
+      Bs[jb][nn] = (n < N && j2 < rl) ? __uint_as_float((uint32_t)B[(long)j2 * N + n] << 16) : 0.0f;
+    }
+    __syncthreads();
+    const int jn = min(kBakeChunk, rl - j0);
+    for (int jj = 0; jj < jn; ++jj) {
+      float a[4], b[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        a[q] = As[jj][tx * 4 + q];
+        b[q] = Bs[jj][ty * 4 + q];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = __fmaf_rn(a[q], b[i], acc[i][q]);
+    }
+    __syncthreads();
   }
-  const float w = __uint_as_float((uint32_t)W[(long)n * K + k] << 16);
-  const __nv_bfloat16 h = __float2bfloat16_rn(__fadd_rn(w, __fmul_rn(scale, acc)));
-  Wb[(long)n * K + k] = *reinterpret_cast<const uint16_t*>(&h);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = n0 + ty * 4 + i;
+    if (n >= N) continue;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k = k0 + tx * 4 + q;
+      if (k >= K) continue;
+      const float w = __uint_as_float((uint32_t)W[(long)n * K + k] << 16);
+      const __nv_bfloat16 h = __float2bfloat16_rn(__fadd_rn(w, __fmul_rn(scale, acc[i][q])));
+      Wb[(long)n * K + k] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_lora_bake(const uint16_t* W, const uint16_t* A, const uint16_t* B, int N, int K, int rl,
                              float scale, uint16_t* Wb, cudaStream_t st) {
-  const dim3 grid((unsigned)((K + 255) / 256), (unsigned)N);
+  const dim3 grid((unsigned)((K + kBakeTile - 1) / kBakeTile), (unsigned)((N + kBakeTile - 1) / kBakeTile));
   lora_bake_kernel<<<grid, 256, 0, st>>>(W, A, B, N, K, rl, scale, Wb);
   return cudaGetLastError();
 }
