@@ -340,6 +340,89 @@ def run_bake(args):
         "gpu_launches": 2 * args.steps}), flush=True)
 
 
+def run_block(args):
+    """The double-stream block at batch 2 (M = 9216, g = 128): fused QKV
+    3072 -> 9216, out-projection 3072 -> 3072, MLP 3072 -> 12288 (GELU fused)
+    -> 3072, all W4A4 with rank 64; the W8A8 first and last projections
+    (3072 -> 3072) and the timestep MLP layer (256 -> 3072 at M = 2).  Each
+    layer runs as its whole-layer call (activation quantization + GEMM);
+    per-layer and whole-block device times."""
+    import torch
+    import w4a4_int4_quantized_b200 as w4
+    from w4a4_int4_quantized_b200 import inputs
+    w4.load_library()
+    names = ["block_first_w8a8", "block_qkv", "block_out", "block_mlp_up", "block_mlp_down", "block_last_w8a8",
+             "block_tmlp_w8a8"]
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    layers = []
+    for nm in names:
+        sp = inputs.WORKLOADS[nm]
+        d = inputs.make_layer(sp)
+        L = dict(spec=sp, X=dev(d["X"]), bias=dev(d["bias"]) if d["bias"] is not None else None,
+                 Y=torch.empty((sp.M, sp.N), dtype=torch.bfloat16, device="cuda"))
+        if sp.w8a8:
+            L["Wq"], L["ws"] = w4.w8a8_quantize_weights(dev(d["W"]), sp.group)
+            L["wsp"] = torch.empty((w4.w8a8_workspace_bytes(sp.M, sp.K),), dtype=torch.uint8, device="cuda")
+        else:
+            L["Wq"], L["ws"] = w4.w4a4_quantize_weights(dev(d["W"]), sp.group)
+            L["L1"], L["L2"] = dev(d["L1"]), dev(d["L2"])
+            L["wsp"] = torch.empty((w4.w4a4_workspace_bytes(sp.M, sp.K, sp.rank),), dtype=torch.uint8,
+                                   device="cuda")
+        layers.append(L)
+
+    def run(L):
+        sp = L["spec"]
+        if sp.w8a8:
+            w4.w8a8_linear(L["X"], L["Wq"], L["ws"], sp.group, L["bias"], Y=L["Y"], workspace=L["wsp"])
+        elif sp.name == "block_mlp_up":
+            w4.w4a4_linear_gelu(L["X"], L["Wq"], L["ws"], sp.group, L["L1"], L["L2"], L["bias"], Y=L["Y"],
+                                workspace=L["wsp"])
+        else:
+            w4.w4a4_linear(L["X"], L["Wq"], L["ws"], sp.group, L["L1"], L["L2"], L["bias"], Y=L["Y"],
+                           workspace=L["wsp"])
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n * 1e3
+
+    per = {L["spec"].name: timed(lambda L=L: run(L), args.steps) for L in layers}
+
+    def block():
+        for L in layers:
+            run(L)
+
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = time.perf_counter()
+    us = timed(block, args.steps)
+    clocks.mark(t0, time.perf_counter())
+    clk = clocks.stop()
+    ops = sum(2.0 * L["spec"].M * L["spec"].N * L["spec"].K for L in layers)
+    err = w4.w4a4_get_device_error()
+    if err:
+        raise SystemExit(f"device error word {err:#x}")
+    print(json.dumps({
+        "metric": "Flux-like double-stream block at batch 2 (M=9216): us per block of linear layers",
+        "value": us, "unit": "us", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3,
+        "tops": ops / (us * 1e-6) / 1e12, "per_layer_us": per,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 / int8 codes (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
+        "config": {"workload": "block_batch2", "M": 9216, "group": 128, "rank": 64},
+        "gpu_launches": sum(2 if L["spec"].w8a8 else 3 for L in layers) * args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -350,6 +433,8 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--block", action="store_true",
+                    help="time the linear layers of the double-stream block at batch 2 (M=9216)")
     ap.add_argument("--bake-lora", type=int, default=0,
                     help="time baking a LoRA of this rank into the weights with stochastic re-quantization")
     ap.add_argument("--mlp", action="store_true",
@@ -363,6 +448,12 @@ def main():
         raise SystemExit("--warmup must be >= 3")
 
     from w4a4_int4_quantized_b200 import inputs
+    if args.block:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the block is measured by the GPU arm only"}))
+            return
+        run_block(args)
+        return
     if args.bake_lora:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the bake is measured by the GPU arm only"}))

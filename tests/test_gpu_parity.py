@@ -400,5 +400,48 @@ def test_mlp_layers_full_size_sampled(name):
     check_output(host_f64(Y)[rows], y_ref, lowrank=True)
 
 
+def test_block_layers_full_size_sampled():
+    """The double-stream block at batch 2 (M=9216): the fused QKV projection
+    (3072 -> 9216, r=64) through w4a4_linear and the W8A8 first projection
+    (3072 -> 3072) through w8a8_linear, on sampled token rows: codes, scales
+    and accumulators bit-exact, outputs within tolerance."""
+    import torch
+    spec = inputs.WORKLOADS["block_qkv"]
+    d = inputs.make_layer(spec)
+    X, W, L1, L2 = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["L1"]), dev_bf16(d["L2"])
+    b = dev_bf16(d["bias"]) if d["bias"] is not None else None
+    Wq, ws = w4.w4a4_quantize_weights(W, spec.group)
+    Y = w4.w4a4_linear(X, Wq, ws, spec.group, L1, L2, b)
+    Xq, xs, T = w4.w4a4_rotate_quantize_act(X, spec.group, L1)
+    acc = torch.empty((spec.M, spec.N), dtype=torch.int32, device="cuda")
+    w4.w4a4_gemm(Xq, xs, Wq, ws, spec.group, T, L2, b, acc_debug=acc)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.random.default_rng(7).choice(spec.M, size=16, replace=False),
+                                     [0, spec.M - 1]]))
+    wp, wsr, wq = oracle.quantize_w4(d["W"], spec.group)
+    assert np.array_equal(Wq.cpu().numpy(), wp) and np.array_equal(ws.cpu().numpy(), wsr)
+    xp, xsr, xq = oracle.quantize_w4(d["X"][rows], spec.group)
+    assert np.array_equal(Xq.cpu().numpy()[rows], xp)
+    acc_ref = oracle.int_gemm(xq, wq)
+    assert np.array_equal(acc.cpu().numpy()[rows], acc_ref)
+    t_ref = oracle.lowrank_down(d["X"][rows], d["L1"])
+    y_ref = oracle.epilogue(acc_ref, xsr, wsr, spec.group, t_ref, d["L2"], d["bias"])
+    check_output(host_f64(Y)[rows], y_ref, lowrank=True)
+
+    spec8 = inputs.WORKLOADS["block_first_w8a8"]
+    d8 = inputs.make_layer(spec8)
+    X8, W8 = dev_bf16(d8["X"]), dev_bf16(d8["W"])
+    b8 = dev_bf16(d8["bias"]) if d8["bias"] is not None else None
+    Wq8, ws8 = w4.w8a8_quantize_weights(W8, spec8.group)
+    Y8 = w4.w8a8_linear(X8, Wq8, ws8, spec8.group, b8)
+    torch.cuda.synchronize()
+    wq8, wsr8 = oracle.quantize_w8(d8["W"], spec8.group)
+    assert np.array_equal(Wq8.cpu().numpy(), wq8) and np.array_equal(ws8.cpu().numpy(), wsr8)
+    xq8, xsr8 = oracle.quantize_w8(d8["X"][rows], spec8.group)
+    acc8 = oracle.int_gemm(xq8, wq8)
+    y8_ref = oracle.epilogue(acc8, xsr8, wsr8, spec8.group, None, None, d8["bias"])
+    check_output(host_f64(Y8)[rows], y8_ref, lowrank=False)
+
+
 def test_no_device_error_after_runs():
     assert w4.w4a4_get_device_error() == 0
