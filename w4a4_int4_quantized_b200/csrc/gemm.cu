@@ -25,12 +25,15 @@
 //   warp 16     TMA: packed A and B tiles (64-byte rows, 64-byte swizzle)
 //               into a shared-memory ring (no multicast), and per tile the
 //               low-rank operand tiles T and L2;
-//   warps 0-7   widen A rows (one row per thread, conflict-free 16-byte
-//               reads) and tcgen05.st them into a TMEM ring -- A is read by
-//               the MMA from tensor memory;
-//   warps 8-15  widen B rows into a ring in the 128-byte-swizzled K-major
-//               layout the MMA reads from shared memory;
-//               (two sets of warps take alternate k-blocks)
+//   warps 0-15  four sets of four warps; set s widens the k-blocks
+//               g = s (mod 4).  Each thread takes one A row and one B row
+//               (conflict-free 16-byte reads): A is tcgen05.st into a TMEM
+//               ring (the MMA reads A from tensor memory), B is stored into
+//               a ring in the 128-byte-swizzled K-major layout the MMA reads
+//               from shared memory.  Each widen is a chain of shared-memory
+//               round trips (stage barrier, loads, release, free-slot
+//               barrier, stores, hand-off), so four chains in flight per CTA
+//               keep pace with the MMAs where two did not;
 //   warp 17     (even CTA) one thread issues the pair MMAs and commits each
 //               stage to the barriers of both CTAs; (odd CTA) relays the
 //               arrival of TMA-only operands to the even CTA.
@@ -69,6 +72,8 @@ constexpr int kTmaWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kWaitWarp = 18;
 constexpr int kIssueBar = 2;     // named barrier: MMA warp + waiter warp
+constexpr int kSets = 4;         // widen sets; set s widens the k-blocks g = s (mod kSets)
+constexpr int kSetWarps = 4;     // warps per set: one A row and one B row per thread
 constexpr int S8 = 5;            // INT8 TMA stages
 constexpr int LRC = 128;         // low-rank rank chunk per MMA round
 constexpr uint32_t kTmemCols = 512;
@@ -85,8 +90,9 @@ constexpr int kBarBytes = 512;
 template <int MODE, bool LR>
 struct Cfg {
   static constexpr bool PACKED = MODE != 0;          // the widen pipeline runs
-  static constexpr int PS = 5;                      // TMA stages (A + packed B)
-  static constexpr int US = MODE == 2 ? 4 : 6;       // widened stages (W4A8: B only)
+  static constexpr int PS = 4;                      // TMA stages (A + packed B), kSets apart
+  static constexpr int US = MODE == 2 ? 4 : 7;       // widened stages (W4A8: B only)
+  static constexpr int kLead = US - 2;               // k-blocks widened ahead of an epilogue
   static constexpr int BN = LR ? 128 : 256;          // N per pair tile
   static constexpr int BNH = BN / 2;                 // B rows staged per CTA
   static constexpr int kARow = MODE == 2 ? BK : BK / 2;  // bytes of an A row per k-block
@@ -113,6 +119,10 @@ struct Cfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kACol0 + US * (BK / 4) <= kTmemCols, "TMEM budget");
   static_assert(PS <= 8 && US <= 8, "barrier arrays");
+  // set s waits on every fill of its own packed stages (g = s mod kSets), in
+  // order, so a phase-parity wait can never match a fill two phases old
+  static_assert(PS % kSets == 0, "each widen set owns its packed stages");
+  static_assert(US >= kSets && kLead >= 1, "widened ring");
   static_assert(kWOff % 1024 == 0, "128-byte swizzle atoms");
   static_assert(!LR || kLrCol + BN <= kACol0, "TMEM budget (low-rank accumulator)");
 };
@@ -248,11 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int s = 0; s < 8; ++s) {
         mbar_init(&bar->tma_full[s], 1);
-        // W4A4: the 8 widen warps of a set read the stage; W4A8: its 4 B
+        // W4A4: the 4 widen warps of a set read the stage; W4A8: the same 4
         // warps plus the MMA commit (the MMA reads A from the stage); W8A8:
         // the MMA commit
-        mbar_init(&bar->tma_empty[s], MODE == 1 ? 8 : (MODE == 2 ? 5 : 1));
-        mbar_init(&bar->full[s], PACKED ? 16 : 1);  // 8 widen warps per CTA, or 1 relay
+        mbar_init(&bar->tma_empty[s], MODE == 1 ? kSetWarps : (MODE == 2 ? kSetWarps + 1 : 1));
+        mbar_init(&bar->full[s], PACKED ? 2 * kSetWarps : 1);  // a set's warps in both CTAs, or 1 relay
         mbar_init(&bar->empty[s], 1);
       }
       mbar_init(&bar->lr_full, 1);
@@ -476,12 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warps 0-7 widen A (TMEM), warps 8-15 widen B (smem); two sets of warps
     // take alternate k-blocks (set 0 even, set 1 odd) so that each warp has
     // two MMA k-blocks of time per widen.  All 16 run the epilogue.
-    const bool is_a = warp < 8;
-    const int set = (warp >> 2) & 1;
+    const int set = warp >> 2;
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;                   // operand row within this CTA's tile
+    const int r = quad * 32 + lane;                   // A row and B row within this CTA's tile
+    const bool has_b = r < BNH;                       // warp-uniform
+    constexpr bool kWidenA = MODE == 1;               // W4A8 reads int8 A straight from the stage
 
-    // widen k-block g of this CTA's A or B rows
+    // widen k-block g: this thread's A row into TMEM and its B row into the
+    // widened shared-memory ring
     auto widen = [&](int g) -> bool {
       const int ps = g % PS;
       const int u = g % US;
@@ -489,47 +501,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         set_device_error(prm.err, kDevErrTimeoutFull);
         return false;
       }
-      if (!is_a && r >= BNH) {
-        // B has only BNH rows per CTA: surplus lanes only take part in the
-        // warp-level hand-offs
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->tma_empty[ps]);
-        if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
-          set_device_error(prm.err, kDevErrTimeoutEmpty);
-          return false;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
-        return true;
-      }
-      constexpr bool kA8 = MODE == 2;
-      if (kA8 && is_a) {
-        // W4A8: the MMA reads this int8 A tile straight from the TMA stage
-        // (released by its commit); the A warps only report, after the
-        // previous use of widened stage u has been consumed, that the tile
-        // has landed in this CTA
-        if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
-          set_device_error(prm.err, kDevErrTimeoutEmpty);
-          return false;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
-        return true;
-      }
-      const uint32_t src = sbase + (uint32_t)(ps * C::kPkStage + (is_a ? 0 : C::kPkA) + r * (BK / 2));
+      const uint32_t stage = sbase + (uint32_t)(ps * C::kPkStage) + (uint32_t)(r * (BK / 2));
       const uint32_t rsw = (uint32_t)((r >> 1) & 3);
-      uint4 pk[4];
+      uint4 pa[4], pb[4];
+      uint32_t seen = 0;
+      if (kWidenA) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) pk[c] = ld_shared_v4(src + ((((uint32_t)c) ^ rsw) << 4));
+        for (int c = 0; c < 4; ++c) {
+          pa[c] = ld_shared_v4(stage + ((((uint32_t)c) ^ rsw) << 4));
+          seen ^= pa[c].x ^ pa[c].y ^ pa[c].z ^ pa[c].w;
+        }
+      }
+      if (has_b) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          pb[c] = ld_shared_v4(stage + (uint32_t)C::kPkA + ((((uint32_t)c) ^ rsw) << 4));
+          seen ^= pb[c].x ^ pb[c].y ^ pb[c].z ^ pb[c].w;
+        }
+      }
       // Hand the packed stage back to TMA only once every lane's loads have
       // returned: the arrive is made data-dependent on all loaded words (an
       // mbarrier arrive by itself does not wait for this warp's outstanding
       // shared-memory loads, and the next bulk copy into the stage would
       // overwrite data not yet read).  Exactly one lane arrives whatever the
       // value.
-      uint32_t seen = 0;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) seen ^= pk[c].x ^ pk[c].y ^ pk[c].z ^ pk[c].w;
       seen = __reduce_or_sync(0xffffffffu, seen);
       if (lane == (seen == 0x9E3779B9u ? 1 : 0)) mbar_arrive(&bar->tma_empty[ps]);
       if (!mbar_wait(&bar->empty[u], ((uint32_t)(g / US) & 1u) ^ 1u)) {
@@ -537,24 +532,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         return false;
       }
       tc_fence_after();
-      if (is_a) {
+      if (kWidenA) {
         uint32_t regs[32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 c0, c1;
-          widen16(pk[c], c0, c1);
+          widen16(pa[c], c0, c1);
           regs[8 * c + 0] = c0.x; regs[8 * c + 1] = c0.y; regs[8 * c + 2] = c0.z; regs[8 * c + 3] = c0.w;
           regs[8 * c + 4] = c1.x; regs[8 * c + 5] = c1.y; regs[8 * c + 6] = c1.z; regs[8 * c + 7] = c1.w;
         }
         tmem_st_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + kACol0 + (uint32_t)(u * (BK / 4)), regs);
-        tmem_wait_st();
-        tc_fence_before();
-      } else {
+      }
+      if (has_b) {
         const uint32_t row =
             sbase + (uint32_t)(PS * C::kPkStage + u * C::kWideB + (r >> 3) * 1024 + (r & 7) * 128);
         const uint32_t rsw128 = (uint32_t)(r & 7);
         uint32_t zk = 0;
-        if constexpr (kA8) {
+        if constexpr (MODE == 2) {
           // zero point of this weight row, as the per-byte bias 128 - z
           const int n = tile_n(g / nk) + (int)rank * BNH + r;
           const uint32_t z = n < p.N ? (uint32_t)__ldg(p.w_zero + n) : 0u;
@@ -563,14 +557,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint4 c0, c1;
-          if constexpr (kA8)
-            widen16_zero_point(pk[c], zk, c0, c1);
+          if constexpr (MODE == 2)
+            widen16_zero_point(pb[c], zk, c0, c1);
           else
-            widen16(pk[c], c0, c1);
+            widen16(pb[c], c0, c1);
           st_shared_v4(row + ((((uint32_t)(2 * c)) ^ rsw128) << 4), c0);
           st_shared_v4(row + ((((uint32_t)(2 * c + 1)) ^ rsw128) << 4), c1);
         }
         fence_proxy_async_smem();
+      }
+      if (kWidenA) {
+        tmem_wait_st();
+        tc_fence_before();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
@@ -674,17 +672,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < my_tiles; ++i) epilogue(i);
     } else {
       // The epilogue of tile i-1 runs before this warp widens any k-block
-      // kb >= min(US, nk) of tile i: the first k-blocks of tile i are then
-      // ready the moment the accumulator is released, and nothing widened
-      // before the epilogue depends on tile i's MMAs.
-      const int lead = min(US, nk);
+      // kb >= min(kLead, nk) of tile i: the first k-blocks of tile i are then
+      // ready the moment the accumulator is released.  kLead < US keeps those
+      // early k-blocks clear of the stages that tile i-1's last MMAs free, so
+      // every warp reaches the epilogue as soon as the accumulator is final.
+      const int lead = min(C::kLead, nk);
       int next_epi = 0;
       int i = 0, kb = set;
       while (kb >= nk) { kb -= nk; ++i; }
-      for (int g = set; g < total_kb; g += 2) {
+      for (int g = set; g < total_kb; g += kSets) {
         while (next_epi < i - 1 || (next_epi == i - 1 && kb >= lead)) epilogue(next_epi++);
         if (!widen(g)) break;
-        kb += 2;
+        kb += kSets;
         while (kb >= nk) { kb -= nk; ++i; }
       }
       while (next_epi < my_tiles) epilogue(next_epi++);
