@@ -115,6 +115,8 @@ GEMM_CASES = [
     (130, 520, 1280, 64, 32, True),
     (257, 768, 3072, 128, 0, True),
     (96, 512, 12288, 128, 128, False),  # long K
+    (300, 640, 1024, 64, 144, False),   # two low-rank chunks, the second 16 ranks
+    (2048, 3072, 256, 128, 256, True),  # rank 256 and more tiles than pairs: buffer hand-off across tiles
 ]
 
 

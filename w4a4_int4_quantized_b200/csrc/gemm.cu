@@ -45,9 +45,11 @@
 //               stores.
 // The kernel is persistent: one pair per TPC walks its output tiles, and the
 // TMA and widen stages run ahead into the next tile while the epilogue of the
-// current one drains the accumulator.  With a low-rank branch the tile is
-// 256 x 128, so that TMEM holds the int32 accumulator, an fp32 accumulator
-// for T L2 (bf16 MMAs issued after each tile's integer MMAs) and the A ring.
+// current one drains the accumulator.  With a low-rank branch the tile stays
+// 256 x 256 and TMEM holds no second accumulator: the epilogue rewrites the
+// int32 accumulator in place as fp32 (acc s_a) s_w', bf16 MMAs accumulate
+// T L2 onto it (operand chunks of 128 ranks staged by TMA), and a second read
+// adds the bias and stores bf16 straight from registers.
 // The INT8 path skips the widening: TMA writes both operands straight into
 // the 128-byte-swizzled layout and the MMA reads both from shared memory.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
@@ -91,9 +93,9 @@ template <int MODE, bool LR>
 struct Cfg {
   static constexpr bool PACKED = MODE != 0;          // the widen pipeline runs
   static constexpr int PS = 4;                      // TMA stages (A + packed B), kSets apart
-  static constexpr int US = MODE == 2 ? 4 : 7;       // widened stages (W4A8: B only)
+  static constexpr int US = MODE == 2 ? 4 : (LR ? 5 : 7);  // widened stages (W4A8: B only)
   static constexpr int kLead = US - 2;               // k-blocks widened ahead of an epilogue
-  static constexpr int BN = LR ? 128 : 256;          // N per pair tile
+  static constexpr int BN = 256;                     // N per pair tile
   static constexpr int BNH = BN / 2;                 // B rows staged per CTA
   static constexpr int kARow = MODE == 2 ? BK : BK / 2;  // bytes of an A row per k-block
   static constexpr int kPkA = BM * kARow;            // A stage (8 KB packed, 16 KB int8)
@@ -106,15 +108,18 @@ struct Cfg {
   static constexpr int kRing = PACKED ? PS * kPkStage + US * kWideB : S8 * kI8Stage;
   static constexpr int kWOff = PS * kPkStage;        // widened B ring
   static constexpr int kLrT = BM * LRC * 2;          // T chunk: 128 rows x 128 ranks, two 64-wide boxes
-  static constexpr int kLrL2 = BNH * LRC * 2;        // L2 chunk: 128 ranks x BNH columns
+  static constexpr int kLrL2 = BNH * LRC * 2;        // L2 chunk: 128 ranks x BNH columns, two 64-wide boxes
   static constexpr int kLrBytes = LR ? kLrT + kLrL2 : 0;
   static constexpr int kVecBytes = 2 * 2 * BN * 4;   // scales + bias, two tiles
   static constexpr int kLrOff = kRing;
   static constexpr int kOutOff = kLrOff + kLrBytes;
-  static constexpr int kVecOff = kOutOff + kOutStageBytes;
+  // the low-rank form stages its bf16 tiles in the operand buffer, free once
+  // the tile's low-rank MMAs have completed
+  static constexpr int kOutBytes = LR ? 0 : kOutStageBytes;
+  static constexpr int kStageOff = LR ? kLrOff : kOutOff;
+  static constexpr int kVecOff = kOutOff + kOutBytes;
   static constexpr int kDataBytes = kVecOff + kVecBytes;
   static constexpr int kSmemBytes = kDataBytes + kBarBytes + 1024;
-  static constexpr uint32_t kLrCol = BN;             // fp32 low-rank accumulator (LR only)
   static constexpr int kColsPerWarp = BN / 4;        // epilogue: 4 warps per TMEM lane quadrant
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kACol0 + US * (BK / 4) <= kTmemCols, "TMEM budget");
@@ -124,7 +129,8 @@ struct Cfg {
   static_assert(PS % kSets == 0, "each widen set owns its packed stages");
   static_assert(US >= kSets && kLead >= 1, "widened ring");
   static_assert(kWOff % 1024 == 0, "128-byte swizzle atoms");
-  static_assert(!LR || kLrCol + BN <= kACol0, "TMEM budget (low-rank accumulator)");
+  static_assert(!LR || MODE == 1, "low-rank branch: W4A4 only");
+  static_assert(!LR || kOutStageBytes <= kLrBytes, "epilogue staging inside the low-rank buffer");
 };
 
 struct Params {
@@ -137,9 +143,12 @@ struct Barriers {
   uint64_t tma_empty[8];
   uint64_t full[8];      // even CTA: a stage is complete in both CTAs
   uint64_t empty[8];
+  uint64_t conv;         // even CTA: both CTAs' epilogues turned the accumulator into fp32
+  uint64_t lr_done;      // the low-rank MMAs of the tile completed
   uint64_t lr_full;      // this CTA's low-rank chunk landed (TMA)
   uint64_t lr_ready;     // even CTA: the odd CTA's low-rank chunk landed (relay)
-  uint64_t lr_empty;     // the low-rank MMAs of the chunk completed
+  uint64_t lr_empty;     // the low-rank MMAs of a chunk (not the tile's last) completed
+  uint64_t lr_free;      // the epilogue's stores staged in the low-rank buffer have been read
   uint64_t acc_full;
   uint64_t acc_empty;    // even CTA: both CTAs' epilogues have read the accumulators
   uint64_t drain;
@@ -265,9 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar->full[s], PACKED ? 2 * kSetWarps : 1);  // a set's warps in both CTAs, or 1 relay
         mbar_init(&bar->empty[s], 1);
       }
+      mbar_init(&bar->conv, 32);       // 16 epilogue warps per CTA
+      mbar_init(&bar->lr_done, 1);
       mbar_init(&bar->lr_full, 1);
       mbar_init(&bar->lr_ready, 1);
       mbar_init(&bar->lr_empty, 1);
+      mbar_init(&bar->lr_free, 16);     // 16 epilogue warps of this CTA
       mbar_init(&bar->acc_full, 1);
       mbar_init(&bar->acc_empty, 32);  // 16 epilogue warps per CTA
       mbar_init(&bar->drain, 1);
@@ -293,14 +305,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kABytes = PACKED ? C::kPkA : C::kI8A;
       constexpr int kColA = PACKED ? C::kARow : BK;   // bytes per k-block of an A / B row
       constexpr int kColB = PACKED ? BK / 2 : BK;
-      int s = 0, lr_n = 0;
+      int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      // Low-rank operand chunks (T rows: K-major, two 64-rank boxes; L2
+      // columns: N-major, two 64-column boxes) go through one buffer, in
+      // order: load q = tile * lr_chunks + chunk.  A load becomes eligible
+      // once its tile's k-blocks are half issued and goes out as soon as the
+      // buffer is free; this thread never blocks on the buffer while k-block
+      // loads remain, since freeing it can depend (through the epilogue) on
+      // widening k-blocks still to be loaded.
+      const int lr_total = my_tiles * lr_chunks;
+      int lr_n = 0, lr_eligible = 0;
+      auto issue_lr = [&]() {
+        const int per_tile = max(lr_chunks, 1);
+        const int ti = lr_n / per_tile, c = lr_n - ti * per_tile;
+        const uint32_t lr = sbase + (uint32_t)C::kLrOff;
+        const int ra = tile_m(ti), rb = tile_n(ti) + (int)rank * BNH;
+        const bool second = p.rank - c * LRC > 64;   // ranks past 64 in this chunk
+        mbar_arrive_expect_tx(&bar->lr_full, (uint32_t)((second ? C::kLrT : C::kLrT / 2) + C::kLrL2));
+        tma_load_2d(lr, &tmT, c * LRC, ra, &bar->lr_full);
+        if (second) tma_load_2d(lr + C::kLrT / 2, &tmT, c * LRC + 64, ra, &bar->lr_full);
+        tma_load_2d(lr + C::kLrT, &tmL2, rb, c * LRC, &bar->lr_full);
+        tma_load_2d(lr + C::kLrT + C::kLrL2 / 2, &tmL2, rb + 64, c * LRC, &bar->lr_full);
+        ++lr_n;
+      };
+      // the buffer is free for load q: after the previous chunk's MMAs (same
+      // tile) or after the previous tile's epilogue stores read their staging
+      auto lr_buffer_free = [&](bool block) -> bool {
+        const int per_tile = max(lr_chunks, 1);
+        const int ti = lr_n / per_tile, c = lr_n - ti * per_tile;
+        if (c == 0 && ti == 0) return true;
+        uint64_t* b = c == 0 ? &bar->lr_free : &bar->lr_empty;
+        const uint32_t parity = (uint32_t)(c == 0 ? ti - 1 : ti * (per_tile - 1) + c - 1) & 1u;
+        return block ? mbar_wait(b, parity) : mbar_try_wait(b, parity);
+      };
+      auto lr_ready_now = [&]() { return LR && lr_n < lr_eligible && lr_buffer_free(false); };
       for (int i = 0; i < my_tiles && ok; ++i) {
         const int row_a = tile_m(i);
         const int row_b = tile_n(i) + (int)rank * BNH;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&bar->tma_empty[s], ph ^ 1u)) {
+          // wait for the stage, issuing any low-rank load that is due
+          bool got = false;
+          const unsigned long long t0 = globaltimer_ns();
+          for (uint32_t it = 0;; ++it) {
+            if (lr_ready_now()) issue_lr();
+            if (mbar_try_wait(&bar->tma_empty[s], ph ^ 1u)) {
+              got = true;
+              break;
+            }
+            if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+          }
+          if (!got) {
             set_device_error(prm.err, kDevErrTimeoutEmpty);
             ok = false;
             break;
@@ -310,24 +366,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst, &tmA, kb * kColA, row_a, &bar->tma_full[s]);
           tma_load_2d(dst + kABytes, &tmB, kb * kColB, row_b, &bar->tma_full[s]);
           if (++s == NS) { s = 0; ph ^= 1u; }
+          if (LR && kb == nk / 2) lr_eligible = (i + 1) * lr_chunks;
         }
-        if (LR) {
-          // low-rank operand chunks of this tile: T rows (K-major, two
-          // 64-rank boxes) and L2 columns (N-major, one 128-rank box)
-          for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
-            if (!mbar_wait(&bar->lr_empty, ((uint32_t)lr_n & 1u) ^ 1u)) {
-              set_device_error(prm.err, kDevErrTimeoutEmpty);
-              ok = false;
-              break;
-            }
-            const uint32_t lr = sbase + (uint32_t)C::kLrOff;
-            const bool second = p.rank - c * LRC > 64;   // ranks past 64 in this chunk
-            mbar_arrive_expect_tx(&bar->lr_full, (uint32_t)((second ? C::kLrT : C::kLrT / 2) + C::kLrL2));
-            tma_load_2d(lr, &tmT, c * LRC, row_a, &bar->lr_full);
-            if (second) tma_load_2d(lr + C::kLrT / 2, &tmT, c * LRC + 64, row_a, &bar->lr_full);
-            tma_load_2d(lr + C::kLrT, &tmL2, row_b, c * LRC, &bar->lr_full);
-          }
+      }
+      // the remaining low-rank loads (no k-block load is left to wait for)
+      while (LR && ok && lr_n < lr_total) {
+        if (!lr_buffer_free(true)) {
+          set_device_error(prm.err, kDevErrTimeoutEmpty);
+          break;
         }
+        issue_lr();
       }
     }
   } else if (warp == kMmaWarp) {
@@ -410,10 +458,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++s == NS) s = 0;
           if (++ps == PS) ps = 0;
         }
+        // the integer product of the tile is complete
+        if (ok && lane == 0) tc_commit_pair_mc(&bar->acc_full, 0x3);
+        __syncwarp();
         if (LR) {
-          // T L2 into the fp32 accumulator: A = T (K-major, 128-byte
-          // swizzle, k-step 16 ranks = 32 bytes), B = L2 (N-major, 128-byte
-          // swizzle, k-step 16 ranks = two 8-row atoms)
+          // Once both epilogues have rewritten the accumulator as fp32
+          // ((acc s_a) s_w' in place), T L2 accumulates onto it: A = T
+          // (K-major, 128-byte swizzle, k-step 16 ranks = 32 bytes), B = L2
+          // (N-major, 128-byte swizzle, two 64-column atoms 16 KB apart,
+          // k-step 16 ranks = two 8-row groups)
           for (int c = 0; c < lr_chunks && ok; ++c) {
             if (named_barrier_or(kIssueBar, 64, false)) {
               ok = false;
@@ -426,15 +479,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int ks = 0; ks < ksteps; ++ks) {
                 const uint32_t a_addr = lr + (uint32_t)((ks >> 2) * (C::kLrT / 2) + (ks & 3) * 32);
                 const uint32_t b_addr = lr + (uint32_t)(C::kLrT + ks * 2048);
-                mma_bf16_ss_pair(tmem + C::kLrCol, smem_desc_kmajor_sw128(a_addr),
-                                 smem_desc_mnmajor_sw128(b_addr, 8192, 1024), idesc_lr, (c | ks) != 0 ? 1u : 0u);
+                mma_bf16_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_addr),
+                                 smem_desc_mnmajor_sw128(b_addr, (uint32_t)(C::kLrL2 / 2), 1024), idesc_lr, 1u);
               }
-              tc_commit_pair_mc(&bar->lr_empty, 0x3);
+              if (c + 1 < lr_chunks) tc_commit_pair_mc(&bar->lr_empty, 0x3);
             }
             __syncwarp();
           }
+          if (ok && lane == 0) tc_commit_pair_mc(&bar->lr_done, 0x3);
         }
-        if (ok && lane == 0) tc_commit_pair_mc(&bar->acc_full, 0x3);
         __syncwarp();
       }
       // drain: every MMA issued so far has completed before teardown
@@ -471,7 +524,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++s == NS) { s = 0; ph ^= 1u; }
         }
         for (int c = 0; c < lr_chunks && ok; ++c, ++lr_n) {
-          const bool late = !mbar_wait(&bar->lr_full, (uint32_t)lr_n & 1u) ||
+          // before the first chunk: both epilogues have converted the accumulator
+          const bool late = (c == 0 && !mbar_wait(&bar->conv, (uint32_t)i & 1u)) ||
+                            !mbar_wait(&bar->lr_full, (uint32_t)lr_n & 1u) ||
                             !mbar_wait(&bar->lr_ready, (uint32_t)lr_n & 1u);
           if (late && lane == 0) set_device_error(prm.err, kDevErrTimeoutFull);
           if (named_barrier_or(kIssueBar, 64, late)) {
@@ -483,9 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 16) {
     // ------------------------------------------------ widen (INT4) + epilogue
-    // warps 0-7 widen A (TMEM), warps 8-15 widen B (smem); two sets of warps
-    // take alternate k-blocks (set 0 even, set 1 odd) so that each warp has
-    // two MMA k-blocks of time per widen.  All 16 run the epilogue.
+    // four sets of four warps; set s widens the k-blocks g = s (mod 4), so
+    // that each warp has four MMA k-blocks of time per widen.  All 16 run
+    // the epilogue.
     const int set = warp >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;                   // A row and B row within this CTA's tile
@@ -576,12 +631,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // epilogue of tile i: each of the 16 warps drains its TMEM lane quadrant's
-    // share of the accumulator columns (and of the low-rank accumulator) into
-    // registers, releases the accumulators to the next tile's MMAs, then
-    // dequantizes, adds the low-rank term and the bias and writes bf16
-    // through TMA stores.
+    // share of the accumulator columns (64) into registers, releases the
+    // accumulator to the next tile's MMAs, then dequantizes, adds the bias and
+    // writes bf16 through TMA stores.  With a low-rank branch it first writes
+    // (acc s_a) s_w' back in place as fp32 and waits for the low-rank MMAs to
+    // add T L2 onto it before the final read.
     const int cq = warp >> 2;                         // column quarter
-    const uint32_t stage_out = sbase + (uint32_t)(C::kOutOff + warp * kStageTile);
+    const uint32_t stage_out = sbase + (uint32_t)(C::kStageOff + warp * kStageTile);
     float* vec_base = reinterpret_cast<float*>(smem_raw + (sbase - raw) + C::kVecOff);
     const uint32_t sw64 = (uint32_t)((lane >> 1) & 3);
     auto epilogue = [&](int i) {
@@ -604,32 +660,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bar->acc_full, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
       tc_fence_after();
       uint32_t v[2][32];
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(cq * C::kColsPerWarp);
-      tmem_ld_32x32b_x32(taddr + kAccCol, v[0]);
-      if (LR)
-        tmem_ld_32x32b_x32(taddr + C::kLrCol, v[1]);
-      else
-        tmem_ld_32x32b_x32(taddr + kAccCol + 32, v[1]);
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(cq * C::kColsPerWarp) + kAccCol;
+      // optional copy of the int32 accumulator (parity checks)
+      auto write_debug = [&](const uint32_t(&vv)[32], int ch) {
+        const int n = n_pair + cq * C::kColsPerWarp + ch * 32;
+        if (!p.acc_debug || !mok || n >= p.N) return;
+        const int nv = min(32, p.N - n);
+        uint4* dd = reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (4 * c < nv)
+            dd[c] = make_uint4((uint32_t)((int)vv[4 * c] >> kShift), (uint32_t)((int)vv[4 * c + 1] >> kShift),
+                               (uint32_t)((int)vv[4 * c + 2] >> kShift), (uint32_t)((int)vv[4 * c + 3] >> kShift));
+      };
+      if constexpr (LR) {
+        // Rewrite the accumulator in place as fp32 (acc s_a) s_w', one
+        // 32-column chunk at a time, let the low-rank MMAs add T L2 onto it,
+        // then read the sum back below.
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int c0 = cq * C::kColsPerWarp + ch * 32;
+          tmem_ld_32x32b_x32(taddr + (uint32_t)(ch * 32), v[ch]);
+          tmem_wait_ld();
+          write_debug(v[ch], ch);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 w4 = *reinterpret_cast<const float4*>(s_sw + c0 + 4 * q);
+            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              v[ch][4 * q + h] =
+                  __float_as_uint(__fmul_rn(__fmul_rn(acc_to_float<true>(v[ch][4 * q + h]), sa), wv[h]));
+          }
+          tmem_st_32x32b_x32(taddr + (uint32_t)(ch * 32), v[ch]);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(&bar->conv, 0);
+        if (!mbar_wait(&bar->lr_done, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
+        tc_fence_after();
+      }
+      tmem_ld_32x32b_x32(taddr, v[0]);
+      tmem_ld_32x32b_x32(taddr + 32, v[1]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(&bar->acc_empty, 0);
-      constexpr int kChunks = LR ? 1 : 2;
 #pragma unroll
-      for (int ch = 0; ch < kChunks; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         const int c0 = cq * C::kColsPerWarp + ch * 32;
         const int n = n_pair + c0;
         if (n >= p.N) continue;  // warp-uniform
-        const int nv = min(32, p.N - n);
+        if constexpr (!LR) write_debug(v[ch], ch);
         uint32_t* vv = v[ch];
-        if (p.acc_debug && mok) {
-          uint4* dd = reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            if (4 * c < nv)
-              dd[c] = make_uint4((uint32_t)((int)vv[4 * c] >> kShift), (uint32_t)((int)vv[4 * c + 1] >> kShift),
-                                 (uint32_t)((int)vv[4 * c + 2] >> kShift), (uint32_t)((int)vv[4 * c + 3] >> kShift));
-        }
         uint32_t o[16];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -641,8 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             const int jj = 4 * q + h;
-            float t = __fmul_rn(__fmul_rn(acc_to_float<MODE == 1>(vv[jj]), sa), wv[h]);
-            if (LR) t = __fadd_rn(t, __uint_as_float(v[1][jj]));
+            const float t = LR ? __uint_as_float(vv[jj])
+                               : __fmul_rn(__fmul_rn(acc_to_float<MODE == 1>(vv[jj]), sa), wv[h]);
             y[h] = __fadd_rn(t, bv[h]);
             if constexpr (ACT) y[h] = gelu_tanh(y[h]);
           }
@@ -665,6 +749,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_2d(&tmY, stage_out, n, m_row0);
           bulk_commit();
         }
+      }
+      if constexpr (LR) {
+        // hand the low-rank buffer back to TMA once the stores have read it
+        if (lane == 0) {
+          bulk_wait_read<0>();
+          mbar_arrive(&bar->lr_free);
+        }
+        __syncwarp();
       }
     };
 
@@ -753,10 +845,10 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   if (LR) {
-    // T [M, r]: 64-rank x 128-row boxes; L2 [r, N]: BNH-column x 128-rank boxes
+    // T [M, r]: 64-rank x 128-row boxes; L2 [r, N]: 64-column x 128-rank boxes
     if (!make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.T, (uint64_t)a.M, (uint64_t)a.rank, 64, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap(&tL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.L2, (uint64_t)a.rank, (uint64_t)a.N, C::BNH, LRC,
+        !make_tmap(&tL2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.L2, (uint64_t)a.rank, (uint64_t)a.N, 64, LRC,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   } else {
