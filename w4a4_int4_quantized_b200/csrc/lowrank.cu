@@ -8,7 +8,7 @@
 // A thin product (N = rank <= 256), so the kernel splits K over a cluster of
 // S CTAs (S <= 8) to put enough SMs on the activations: each CTA streams a
 // 128-row tile of X (K-major, 128-byte swizzle) and the matching rows of L1
-// (N-major, 128-byte swizzle) through a 4-deep TMA ring and accumulates its K
+// (N-major, 128-byte swizzle) through a 4- to 8-deep TMA ring and accumulates its K
 // slice with tcgen05.mma kind::f16 into TMEM.  The fp32 partials are drained
 // into each CTA's shared memory and reduced through distributed shared memory
 // in a fixed CTA order (deterministic, no global scratch); each CTA writes
@@ -28,28 +28,30 @@ namespace {
 
 constexpr int BM = 128;        // rows of X per tile
 constexpr int BKL = 64;        // K per stage (128 bytes of bf16: one swizzle row)
-constexpr int NST = 4;         // TMA stages
+constexpr int NSTMAX = 8;      // TMA stages (as many as fit: 4 to 8)
 constexpr int kThreads = 128;
 
 struct LrBarriers {
-  uint64_t full[NST];
-  uint64_t empty[NST];
+  uint64_t full[NSTMAX];
+  uint64_t empty[NSTMAX];
   uint64_t acc_full;
   uint32_t tmem_base;
 };
 
 struct LrParams {
   uint16_t* T;
-  int M, K, r, S;
+  int M, K, r, S, nst;
   unsigned int* err;
 };
 
+// A 16-byte load from a cluster peer's shared memory, without a compiler
+// memory barrier, so that independent loads can be in flight together (the
+// partials are not written again before the kernel's closing cluster barrier).
 __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr)
-               : "memory");
+               : "r"(addr));
   return v;
 }
 
@@ -70,6 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kBB = rb * BKL * 128;                       // L1 stage: rb boxes of 64 K-rows x 128 bytes
   const int kStage = kAB + kBB;
   const int part_pitch = p.r * 4 + 16;                  // fp32 partial row pitch (padded)
+  const int NST = p.nst;
   const int data = max(NST * kStage, BM * part_pitch);
   LrBarriers* bar = reinterpret_cast<LrBarriers*>(smem_raw + (sbase - raw) + data);
 
@@ -173,19 +176,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();
 
   // --------------------------------------------- reduce across the cluster
+  // All S remote loads of an item are issued before any is used (a load
+  // from another CTA's shared memory takes hundreds of cycles); the sum then
+  // runs in CTA order 0 .. S-1, so T does not depend on timing.
   const int rows_per = BM / S;
   const int vec_per_row = p.r / 4;
   for (int item = threadIdx.x; item < rows_per * vec_per_row; item += kThreads) {
     const int rr = (int)crank * rows_per + item / vec_per_row;
     const int c = (item % vec_per_row) * 4;
     const uint32_t local = sbase + (uint32_t)(rr * part_pitch + c * 4);
+    uint4 w[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < S) w[s] = ld_cluster_v4(map_to_rank(local, (uint32_t)s));
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < S; ++s) {
-      const uint4 w = ld_cluster_v4(map_to_rank(local, (uint32_t)s));
-      acc[0] = __fadd_rn(acc[0], __uint_as_float(w.x));
-      acc[1] = __fadd_rn(acc[1], __uint_as_float(w.y));
-      acc[2] = __fadd_rn(acc[2], __uint_as_float(w.z));
-      acc[3] = __fadd_rn(acc[3], __uint_as_float(w.w));
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      if (s < S) {
+        acc[0] = __fadd_rn(acc[0], __uint_as_float(w[s].x));
+        acc[1] = __fadd_rn(acc[1], __uint_as_float(w[s].y));
+        acc[2] = __fadd_rn(acc[2], __uint_as_float(w[s].z));
+        acc[3] = __fadd_rn(acc[3], __uint_as_float(w[s].w));
+      }
     }
     const long m = (long)m0 + rr;
     if (m < p.M) {
@@ -241,17 +253,53 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int m_tiles = (M + BM - 1) / BM;
   const int nkb = K / BKL;
-  int S = 1;
-  while (S < 8 && m_tiles * S * 2 <= sms && S * 2 <= nkb) S *= 2;   // about one CTA per SM
   const int rb = (r + 63) / 64;
   const int stage = BM * BKL * 2 + rb * BKL * 128;
-  const int data = std::max(NST * stage, BM * (r * 4 + 16));
+  // as deep a ring as fits beside the barriers (X streams from HBM once)
+  const int nst = std::max(4, std::min(NSTMAX, (232448 - 2048) / stage));
+  const int data = std::max(nst * stage, BM * (r * 4 + 16));
   const int smem = data + (int)sizeof(LrBarriers) + 1024;
   static int attr_smem[64] = {0};
   if (dev < 64 && attr_smem[dev] < smem) {
     e = cudaFuncSetAttribute(lowrank_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e != cudaSuccess) return e;
     attr_smem[dev] = 232448;
+  }
+  // K split S: the largest power of two (<= 8) for which every cluster of
+  // the grid is resident at once.  Clusters must fit inside one GPC, so the
+  // count that fits is below sms / S for S = 4 and 8; a grid past it runs a
+  // second wave and doubles the time.
+  static int cache_key[64][3];
+  static int cache_s[64] = {0};
+  int S = 0;
+  if (dev < 64 && cache_s[dev] && cache_key[dev][0] == m_tiles && cache_key[dev][1] == nkb &&
+      cache_key[dev][2] == smem)
+    S = cache_s[dev];
+  if (!S) {
+    S = 1;
+    for (int sc = 2; sc <= 8 && sc <= nkb && m_tiles * sc <= sms; sc *= 2) {
+      cudaLaunchConfig_t qc = {};
+      qc.gridDim = dim3(m_tiles * sc, 1, 1);
+      qc.blockDim = dim3(kThreads, 1, 1);
+      qc.dynamicSmemBytes = smem;
+      cudaLaunchAttribute qa;
+      qa.id = cudaLaunchAttributeClusterDimension;
+      qa.val.clusterDim.x = sc;
+      qa.val.clusterDim.y = 1;
+      qa.val.clusterDim.z = 1;
+      qc.attrs = &qa;
+      qc.numAttrs = 1;
+      int max_clusters = 0;
+      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, lowrank_down_kernel, &qc)) != cudaSuccess) return e;
+      if (m_tiles > max_clusters) break;
+      S = sc;
+    }
+    if (dev < 64) {
+      cache_key[dev][0] = m_tiles;
+      cache_key[dev][1] = nkb;
+      cache_key[dev][2] = smem;
+      cache_s[dev] = S;
+    }
   }
   CUtensorMap tX, tL1;
   if (!tmap_bf16(&tX, X, (uint64_t)M, (uint64_t)K, BKL, BM) ||
@@ -271,7 +319,7 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  LrParams prm{T, M, K, r, S, err};
+  LrParams prm{T, M, K, r, S, nst, err};
   e = cudaLaunchKernelEx(&cfg, lowrank_down_kernel, prm, tX, tL1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
