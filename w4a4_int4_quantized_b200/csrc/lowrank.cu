@@ -6,13 +6,13 @@
 // fp32 and is stored as bf16 for the up-projection folded into the GEMM.
 //
 // A thin product (N = rank <= 256), so the kernel splits K over a cluster of
-// S CTAs (S <= 8) to put enough SMs on the activations: each CTA streams a
+// S CTAs (2 <= S <= 8, any size) to put enough SMs on the activations: each CTA streams a
 // 128-row tile of X (K-major, 128-byte swizzle) and the matching rows of L1
 // (N-major, 128-byte swizzle) through a 4- to 8-deep TMA ring and accumulates its K
 // slice with tcgen05.mma kind::f16 into TMEM.  The fp32 partials are drained
 // into each CTA's shared memory and reduced through distributed shared memory
-// in a fixed CTA order (deterministic, no global scratch); each CTA writes
-// 128/S rows of T.
+// in a fixed CTA order (deterministic, no global scratch); CTA c writes rows
+// [c*128/S, (c+1)*128/S) of the tile of T.
 #include <algorithm>
 
 #include <cuda.h>
@@ -179,10 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // All S remote loads of an item are issued before any is used (a load
   // from another CTA's shared memory takes hundreds of cycles); the sum then
   // runs in CTA order 0 .. S-1, so T does not depend on timing.
-  const int rows_per = BM / S;
+  const int row0 = (int)crank * BM / S, row1 = ((int)crank + 1) * BM / S;   // this CTA's rows of T
   const int vec_per_row = p.r / 4;
-  for (int item = threadIdx.x; item < rows_per * vec_per_row; item += kThreads) {
-    const int rr = (int)crank * rows_per + item / vec_per_row;
+  for (int item = threadIdx.x; item < (row1 - row0) * vec_per_row; item += kThreads) {
+    const int rr = row0 + item / vec_per_row;
     const int c = (item % vec_per_row) * 4;
     const uint32_t local = sbase + (uint32_t)(rr * part_pitch + c * 4);
     uint4 w[8];
@@ -265,9 +265,9 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
     if (e != cudaSuccess) return e;
     attr_smem[dev] = 232448;
   }
-  // K split S: the largest power of two (<= 8) for which every cluster of
+  // K split S (cluster size): the largest S <= 8 for which every cluster of
   // the grid is resident at once.  Clusters must fit inside one GPC, so the
-  // count that fits is below sms / S for S = 4 and 8; a grid past it runs a
+  // count that fits is below sms / S for the larger S; a grid past it runs a
   // second wave and doubles the time.
   static int cache_key[64][3];
   static int cache_s[64] = {0};
@@ -277,7 +277,8 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
     S = cache_s[dev];
   if (!S) {
     S = 1;
-    for (int sc = 2; sc <= 8 && sc <= nkb && m_tiles * sc <= sms; sc *= 2) {
+    for (int sc = std::min(8, nkb); sc >= 2 && S == 1; --sc) {
+      if (m_tiles * sc > sms) continue;
       cudaLaunchConfig_t qc = {};
       qc.gridDim = dim3(m_tiles * sc, 1, 1);
       qc.blockDim = dim3(kThreads, 1, 1);
@@ -291,8 +292,7 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
       qc.numAttrs = 1;
       int max_clusters = 0;
       if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, lowrank_down_kernel, &qc)) != cudaSuccess) return e;
-      if (m_tiles > max_clusters) break;
-      S = sc;
+      if (m_tiles <= max_clusters) S = sc;
     }
     if (dev < 64) {
       cache_key[dev][0] = m_tiles;
