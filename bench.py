@@ -42,8 +42,8 @@ HBM_NOMINAL_GBS = 8000.0
 # they were taken from (sha256 prefix); reported as null once the source
 # changes.
 MEASURED_TRAFFIC = {
-    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "72d24aa999c60378", 11.880448e6 + 0.030464e6),
-    "gemm_w4a8": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "72d24aa999c60378", 18.960384e6 + 0.091648e6),
+    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6488a2c765a2d4a6", 11.880448e6 + 0.030464e6),
+    "gemm_w4a8": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6488a2c765a2d4a6", 18.960384e6 + 0.091648e6),
     "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "61d3e84e299a0ca7", 28.377344e6),
 }
 

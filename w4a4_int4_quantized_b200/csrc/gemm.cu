@@ -19,8 +19,8 @@
 // shift of the int32 accumulator (|acc| <= 64 K << 2^23 for K <= 32768).
 //
 // Work decomposition: a cluster of two CTAs (one per SM of a TPC) owns a
-// 256 x BN output tile and issues the pair form of the MMA (cta_group::2):
-// each CTA holds 128 rows of A, BN/2 rows (N) of B and its 128 x BN int32
+// 256 x 256 output tile and issues the pair form of the MMA (cta_group::2):
+// each CTA holds 128 rows of A, 128 rows (N) of B and its 128 x 256 int32
 // accumulator.  Per CTA (k-block = 128 codes):
 //   warp 16     TMA: packed A and B tiles (64-byte rows, 64-byte swizzle)
 //               into a shared-memory ring (no multicast), and per tile the
@@ -49,7 +49,7 @@
 // 256 x 256 and TMEM holds no second accumulator: the epilogue rewrites the
 // int32 accumulator in place as fp32 (acc s_a) s_w', bf16 MMAs accumulate
 // T L2 onto it (operand chunks of 128 ranks staged by TMA), and a second read
-// adds the bias and stores bf16 straight from registers.
+// adds the bias; bf16 tiles leave via TMA stores staged in the operand buffer.
 // The INT8 path skips the widening: TMA writes both operands straight into
 // the 128-byte-swizzled layout and the MMA reads both from shared memory.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
