@@ -280,13 +280,45 @@ w4a4_status w4a4_bake_lora_sr(const void* W, const void* A, const void* B, int l
                               int K, int group, unsigned long long seed, void* W_baked, uint8_t* Wq, float* w_scale,
                               w4a4_stream_t stream);
 
+/* ---------------------------------------------------------------- planning */
+/* Host-only view of how the rotate + quantize kernel is launched, for tools
+ * and for testing the launch-plan caches from many host threads: no CUDA
+ * call is made and nothing is launched.  Given M, K and group (rules as
+ * w4a4_rotate_quantize_act), a device with `sms` SMs on which
+ * `resident_per_sm` CTAs fit, writes shape[4] = {rows per block, threads per
+ * CTA, dynamic shared memory bytes, grid size}.  cached != 0 goes through a
+ * small shared plan cache (the same cache type the launchers use, guarded by
+ * a mutex), cached == 0 computes the plan directly; both give the same
+ * answer.  The pages have no counterpart. */
+w4a4_status w4a4_plan_rotate_quantize(int M, int K, int group, int sms, int resident_per_sm, int cached,
+                                      int* shape);
+
 /* ---------------------------------------------------------------- failures */
 /* Kernels never trap: a wait on another part of the kernel that runs past its
  * time limit (2 s) records a code in a per-device error word and lets the
  * kernel finish.  This call synchronises `stream`, reads the word of the
  * current device into *code (may be NULL), clears it, and returns
- * W4A4_ERR_DEVICE_TIMEOUT when it was non-zero, W4A4_OK otherwise. */
+ * W4A4_ERR_DEVICE_TIMEOUT when it was non-zero, W4A4_OK otherwise.  The code
+ * is an OR of the W4A4_DEVERR_* bits below.  The pages describe no failure
+ * handling for the kernels; this is the library's own. */
+#define W4A4_DEVERR_WAIT_OPERANDS 1u /* a tensor-core issuer gave up waiting for its operands */
+#define W4A4_DEVERR_WAIT_SLOT 2u     /* a producer gave up waiting for a free pipeline stage */
+#define W4A4_DEVERR_WAIT_ACCUM 4u    /* an epilogue gave up waiting for its accumulator */
+#define W4A4_DEVERR_WAIT_DRAIN 8u    /* the final drain of in-flight tensor-core work ran out */
 w4a4_status w4a4_get_device_error(w4a4_stream_t stream, unsigned int* code);
+
+/* Self-test of the bounded waits, for callers that want to see the failure
+ * path work on their device without faulting it.  Launches the low-rank
+ * down-projection of w4a4_rotate_quantize_act (X bf16 [M, K], L1 bf16
+ * [K, rank], T out bf16 [M, rank]; shape and alignment rules as there, rank
+ * > 0) with its operand producer withholding every load and the operand wait
+ * limited to timeout_us microseconds (1 .. 1000000).  The tensor-core issuer's
+ * first wait then runs out: no copy or MMA is in flight when it gives up, the
+ * kernel finishes normally, T is left undefined, and the device error word
+ * afterwards holds W4A4_DEVERR_WAIT_OPERANDS (w4a4_get_device_error returns
+ * W4A4_ERR_DEVICE_TIMEOUT and clears it).  Later calls are unaffected. */
+w4a4_status w4a4_selftest_wait_timeout(const void* X, const void* L1, int M, int K, int rank, void* T,
+                                       unsigned int timeout_us, w4a4_stream_t stream);
 
 #ifdef __cplusplus
 }

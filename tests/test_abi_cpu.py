@@ -219,3 +219,48 @@ def test_valid_call_without_gpu_fails_loudly(lib):
     assert lib.w4a4_quantize_weights(A, 64, 256, 64, B, C, NUL) in (CUDA, DEVICE)
     with pytest.raises(w4.W4A4Error):
         w4._check("w4a4_quantize_weights", lib.w4a4_quantize_weights(A, 64, 256, 64, B, C, NUL))
+
+
+def test_selftest_wait_timeout_validation(lib):
+    f = lib.w4a4_selftest_wait_timeout
+    assert f(NUL, B, 64, 256, 16, C, 1000, NUL) == INVALID
+    assert f(A, NUL, 64, 256, 16, C, 1000, NUL) == INVALID
+    assert f(A, B, 64, 256, 16, NUL, 1000, NUL) == INVALID
+    assert f(A, B, 64, 256, 16, C, 0, NUL) == INVALID          # no wait limit
+    assert f(A, B, 64, 256, 16, C, 2000000, NUL) == INVALID    # over one second
+    assert f(A, B, 64, 256, 0, C, 1000, NUL) == SHAPE          # needs a low-rank branch
+    assert f(A, B, 64, 256, 24, C, 1000, NUL) == SHAPE         # rank not a multiple of 16
+    assert f(A, B, 0, 256, 16, C, 1000, NUL) == SHAPE
+    assert f(A, B, 64, 200, 16, C, 1000, NUL) == SHAPE
+    assert f(ODD, B, 64, 256, 16, C, 1000, NUL) == MISALIGNED
+
+
+def test_device_error_bits_match_the_header():
+    text = open(HEADER).read()
+    bits = dict(re.findall(r"#define W4A4_DEVERR_(\w+) (\d+)u", text))
+    assert {k: int(v) for k, v in bits.items()} == {
+        "WAIT_OPERANDS": w4.DEVERR_WAIT_OPERANDS, "WAIT_SLOT": w4.DEVERR_WAIT_SLOT,
+        "WAIT_ACCUM": w4.DEVERR_WAIT_ACCUM, "WAIT_DRAIN": w4.DEVERR_WAIT_DRAIN}
+
+
+def test_launch_plan_cache_under_host_threads(lib):
+    """The launch-plan cache hands every thread the plan of the shape it asked
+    for while other threads insert and evict other shapes (no CUDA call)."""
+    import concurrent.futures as cf
+    import random
+    shapes = [(m, k, g) for m in (1, 2, 37, 256, 1000, 4608, 9216, 16384)
+              for k in (256, 3072, 12288) for g in (64, 128)]
+    expect = {sh: w4.w4a4_plan_rotate_quantize(*sh, cached=False) for sh in shapes}
+    assert expect[(4608, 3072, 128)] == (4, 96, 4 * 24 * 272 * 2, 592)
+
+    def worker(seed):
+        rnd = random.Random(seed)
+        bad = 0
+        for _ in range(4000):
+            sh = rnd.choice(shapes)
+            if w4.w4a4_plan_rotate_quantize(*sh, cached=True) != expect[sh]:
+                bad += 1
+        return bad
+
+    with cf.ThreadPoolExecutor(8) as ex:
+        assert sum(ex.map(worker, range(8))) == 0

@@ -23,7 +23,8 @@ __all__ = [
     "w8a8_quantize_weights", "w8a8_rotate_quantize_act", "w8a8_gemm", "w8a8_linear",
     "w8a8_workspace_bytes", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear", "w4a8_workspace_bytes",
     "w4a4_lora_merge", "w4a4_gemm_gelu", "w4a4_linear_gelu", "w4a4_mlp", "w4a4_mlp_workspace_bytes",
-    "w4a4_bake_lora_sr", "w4a4_get_device_error",
+    "w4a4_bake_lora_sr", "w4a4_get_device_error", "w4a4_selftest_wait_timeout", "w4a4_plan_rotate_quantize",
+    "DEVERR_WAIT_OPERANDS", "DEVERR_WAIT_SLOT", "DEVERR_WAIT_ACCUM", "DEVERR_WAIT_DRAIN",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +32,8 @@ _LIB_PATH = os.path.join(_HERE, "libw4a4.so")
 _lib = None
 
 W4A4_OK = 0
+# bits of the device error word (W4A4_DEVERR_* in include/w4a4.h)
+DEVERR_WAIT_OPERANDS, DEVERR_WAIT_SLOT, DEVERR_WAIT_ACCUM, DEVERR_WAIT_DRAIN = 1, 2, 4, 8
 STATUS = {
     0: "W4A4_OK", 1: "W4A4_ERR_INVALID_ARG", 2: "W4A4_ERR_UNSUPPORTED_SHAPE", 3: "W4A4_ERR_MISALIGNED",
     4: "W4A4_ERR_CUDA", 5: "W4A4_ERR_DEVICE_TIMEOUT", 6: "W4A4_ERR_UNSUPPORTED_DEVICE", 7: "W4A4_ERR_WORKSPACE",
@@ -82,6 +85,8 @@ def load_library():
         "w4a4_bake_lora_sr": ([P, P, P, I, ctypes.c_float, I, I, I, ctypes.c_ulonglong, P, P, P, P], S),
         "w4a4_mlp": ([P, I, I, I, I, P, P, P, P, I, P, P, P, P, P, I, P, P, P, Z, P], S),
         "w4a4_get_device_error": ([P, ctypes.POINTER(ctypes.c_uint)], S),
+        "w4a4_selftest_wait_timeout": ([P, P, I, I, I, P, ctypes.c_uint, P], S),
+        "w4a4_plan_rotate_quantize": ([I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)], S),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -379,3 +384,26 @@ def w4a4_get_device_error(stream=None) -> int:
     if status not in (0, 5):
         raise W4A4Error("w4a4_get_device_error", status)
     return int(code.value)
+
+
+def w4a4_selftest_wait_timeout(X, L1, timeout_us=1000, T=None, stream=None):
+    """Run the low-rank down-projection with its operand loads withheld and the
+    operand wait limited to `timeout_us`: the wait runs out, the kernel ends
+    normally and the device error word then holds DEVERR_WAIT_OPERANDS.
+    Returns T (undefined contents)."""
+    import torch
+    M, K = X.shape
+    rank = L1.shape[1]
+    T = _empty((M, rank), torch.bfloat16, X) if T is None else T
+    _check("w4a4_selftest_wait_timeout", load_library().w4a4_selftest_wait_timeout(
+        _ptr(X), _ptr(L1), M, K, rank, _ptr(T), timeout_us, _stream(stream)))
+    return T
+
+
+def w4a4_plan_rotate_quantize(M, K, group, sms=148, resident_per_sm=4, cached=True):
+    """Launch shape the rotate + quantize kernel would use (host only, no CUDA
+    call): (rows per block, threads, dynamic shared memory, grid)."""
+    out = (ctypes.c_int * 4)()
+    _check("w4a4_plan_rotate_quantize", load_library().w4a4_plan_rotate_quantize(
+        M, K, group, sms, resident_per_sm, 1 if cached else 0, out))
+    return tuple(out)

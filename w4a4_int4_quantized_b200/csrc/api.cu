@@ -3,6 +3,7 @@
 #include <atomic>
 #include <cstdint>
 
+#include "common.cuh"
 #include "kernels.h"
 #include "w4a4.h"
 
@@ -77,6 +78,10 @@ unsigned int* device_error_word() {
 }  // namespace w4a4
 
 using namespace w4a4;
+
+static_assert(kDevErrTimeoutFull == W4A4_DEVERR_WAIT_OPERANDS && kDevErrTimeoutEmpty == W4A4_DEVERR_WAIT_SLOT &&
+                  kDevErrTimeoutAcc == W4A4_DEVERR_WAIT_ACCUM && kDevErrTimeoutDrain == W4A4_DEVERR_WAIT_DRAIN,
+              "device error bits of the public header");
 
 extern "C" {
 
@@ -374,7 +379,33 @@ w4a4_status w4a4_bake_lora_sr(const void* W, const void* A, const void* B, int l
                                                seed, st));
 }
 
+// ------------------------------------------------------------------ planning
+w4a4_status w4a4_plan_rotate_quantize(int M, int K, int group, int sms, int resident_per_sm, int cached,
+                                      int* shape) {
+  if (!shape) return W4A4_ERR_INVALID_ARG;
+  if (M < 1 || sms < 1 || resident_per_sm < 1) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  const w4a4_status s = check_k_group(K, group);
+  if (s != W4A4_OK) return s;
+  return plan_rotate_quantize_shape(M, K, group, sms, resident_per_sm, cached != 0, shape) ? W4A4_OK
+                                                                                           : W4A4_ERR_UNSUPPORTED_SHAPE;
+}
+
 // ------------------------------------------------------------------ failures
+w4a4_status w4a4_selftest_wait_timeout(const void* X, const void* L1, int M, int K, int rank, void* T,
+                                       unsigned int timeout_us, w4a4_stream_t stream) {
+  if (!X || !L1 || !T) return W4A4_ERR_INVALID_ARG;
+  if (timeout_us < 1 || timeout_us > 1000000) return W4A4_ERR_INVALID_ARG;
+  w4a4_status s = check_rank(rank);
+  if (s != W4A4_OK) return s;
+  if (rank == 0 || M < 1) return W4A4_ERR_UNSUPPORTED_SHAPE;
+  if ((s = check_k_group(K, 128)) != W4A4_OK) return s;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(T)) return W4A4_ERR_MISALIGNED;
+  if ((s = check_device()) != W4A4_OK) return s;
+  return cuda_status(launch_lowrank_down_ex(static_cast<const uint16_t*>(X), static_cast<const uint16_t*>(L1), M, K,
+                                            rank, static_cast<uint16_t*>(T), 1000ull * timeout_us, 1,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 w4a4_status w4a4_get_device_error(w4a4_stream_t stream, unsigned int* code) {
   w4a4_status s = check_device();
   if (s != W4A4_OK) return s;

@@ -10,7 +10,7 @@ namespace w4a4 {
 
 // Codes OR-ed into the library's device error word (passed to kernels as a
 // pointer) when a bounded wait gives up; read and cleared on the host by
-// w4a4_get_device_error().
+// w4a4_get_device_error() (the W4A4_DEVERR_* bits of the public header).
 enum : unsigned int {
   kDevErrTimeoutFull = 1u,      // an MMA issuer waited too long for operands
   kDevErrTimeoutEmpty = 2u,     // a producer waited too long for a free stage
@@ -62,13 +62,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (without trapping) after kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// (without trapping) after limit_ns (kWaitTimeoutNs unless a caller, such as
+// the wait-timeout self-test, passes a shorter limit).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u && globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -62,6 +62,8 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "plan_cache.h"
+#include "tmap.h"
 
 namespace w4a4 {
 
@@ -793,44 +795,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      f = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }();
-  return fn;
-}
-
-// Row-major matrix [rows, cols] of 1- or 2-byte elements as a 2-D tensor map
-// with a (box_cols x box_rows) box; elements past the ends read as zero.
-bool make_tmap(CUtensorMap* tm, CUtensorMapDataType dt, int esize, const void* base, uint64_t rows,
-               uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * (uint64_t)esize};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE, bool LR, bool ACT = false>
 cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   using C = Cfg<MODE, LR>;
   auto kern = gemm_kernel<MODE, LR, ACT>;
-  static int configured[64] = {0};
+  static DeviceFlags configured;   // one per instantiation
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 64 && !configured[dev]) {
+  if (!configured.done(dev)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured[dev] = 1;
+    configured.set(dev);
   }
   CUtensorMap tA, tB, tY, tT, tL2;
   // packed 4-bit rows: 64-byte boxes, 64-byte swizzle; int8 rows: 128-byte
@@ -856,13 +832,8 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
     tL2 = tY;
   }
   const int pairs = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + C::BN - 1) / C::BN);
-  static int sm_count[64] = {0};
-  if (dev < 64 && !sm_count[dev]) {
-    int n = 0;
-    if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    sm_count[dev] = n;
-  }
-  const int sms = dev < 64 ? sm_count[dev] : 148;
+  int sms = 0;
+  if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * std::min(pairs, sms / 2), 1, 1);   // persistent: one pair per TPC
   cfg.blockDim = dim3(kThreads, 1, 1);

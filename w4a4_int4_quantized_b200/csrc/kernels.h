@@ -11,6 +11,10 @@ namespace w4a4 {
 cudaError_t launch_rotate_quantize(const uint16_t* X, int rows, int K, int group, int qmax, uint8_t* out,
                                    float* scale, uint8_t* zero, cudaStream_t st);
 
+// Host-only planning of the rotate + quantize launch shape (no CUDA call):
+// out = {rows per block, threads, dynamic shared memory, grid}.
+bool plan_rotate_quantize_shape(int M, int K, int group, int sms, int resident_per_sm, bool cached, int out[4]);
+
 struct GemmArgs {
   const uint8_t* A;        // activation codes [M, K/2] packed or [M, K] int8
   const float* a_scale;    // [M]
@@ -37,6 +41,12 @@ cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st);
 // T[M, r] (bf16) = X[M, K] (bf16) x L1[K, r] (bf16), fp32 accumulation.
 cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
                                 cudaStream_t st);
+
+// The same with an explicit limit for every bounded wait and, for the
+// wait-timeout self-test, a producer that withholds every operand load (the
+// consumer's first wait then runs out after wait_ns; T is left undefined).
+cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
+                                   unsigned long long wait_ns, int withhold, cudaStream_t st);
 
 // Symmetric INT4 codes of rotated rows with stochastic rounding: q =
 // clamp(floor(y / s + u), -8, 7), u from Philox4x64-10 keyed by `seed`.

@@ -21,6 +21,8 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "plan_cache.h"
+#include "tmap.h"
 
 namespace w4a4 {
 
@@ -42,6 +44,8 @@ struct LrParams {
   uint16_t* T;
   int M, K, r, S, nst;
   unsigned int* err;
+  unsigned long long wait_ns;   // limit of the operand and free-slot waits
+  int withhold;                 // self-test: the producer issues no operand load
 };
 
 // A 16-byte load from a cluster peer's shared memory, without a compiler
@@ -113,10 +117,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------- TMA
+    // (self-test: with `withhold` set nothing is issued, so the MMA thread's
+    // first operand wait runs out; no copy or MMA is then in flight)
     int s = 0;
     uint32_t ph = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(&bar->empty[s], ph ^ 1u)) {
+    for (int kb = kb0; kb < (p.withhold ? kb0 : kb1); ++kb) {
+      if (!mbar_wait(&bar->empty[s], ph ^ 1u, p.wait_ns)) {
         set_device_error(p.err, kDevErrTimeoutEmpty);
         break;
       }
@@ -133,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s = 0;
     uint32_t ph = 0;
     for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(&bar->full[s], ph)) {
+      if (!mbar_wait(&bar->full[s], ph, p.wait_ns)) {
         set_device_error(p.err, kDevErrTimeoutFull);
         break;
       }
@@ -152,6 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // --------------------------------------------- drain partials to smem
   __syncwarp();   // lanes 0 of warps 0 and 1 rejoin before the warp-wide TMEM loads
+  // (always the full limit: the commit that completes this barrier must be
+  // observed before the CTA exits, also after a shortened operand wait)
   if (!mbar_wait(&bar->acc_full, 0)) set_device_error(p.err, kDevErrTimeoutAcc);
   tc_fence_after();
   const int row = warp * 32 + lane;
@@ -214,43 +222,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_lr() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      f = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }();
-  return fn;
-}
-
-bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-               uint32_t box_rows) {
-  auto fn = encode_fn_lr();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 unsigned int* device_error_word();
 
-cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
-                                cudaStream_t st) {
+cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
+                                   unsigned long long wait_ns, int withhold, cudaStream_t st) {
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorInvalidDevicePointer;
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
   const int m_tiles = (M + BM - 1) / BM;
   const int nkb = K / BKL;
   const int rb = (r + 63) / 64;
@@ -259,25 +242,25 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
   const int nst = std::max(4, std::min(NSTMAX, (232448 - 2048) / stage));
   const int data = std::max(nst * stage, BM * (r * 4 + 16));
   const int smem = data + (int)sizeof(LrBarriers) + 1024;
-  static int attr_smem[64] = {0};
-  if (dev < 64 && attr_smem[dev] < smem) {
+  static DeviceFlags attr_set;
+  if (!attr_set.done(dev)) {
     e = cudaFuncSetAttribute(lowrank_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e != cudaSuccess) return e;
-    attr_smem[dev] = 232448;
+    attr_set.set(dev);
   }
   // K split S (cluster size): the largest S <= 8 for which every cluster of
   // the grid is resident at once.  Clusters must fit inside one GPC, so the
   // count that fits is below sms / S for the larger S; a grid past it runs a
   // second wave and doubles the time.
-  static int cache_key[64][3];
-  static int cache_s[64] = {0};
-  int S = 0;
-  if (dev < 64 && cache_s[dev] && cache_key[dev][0] == m_tiles && cache_key[dev][1] == nkb &&
-      cache_key[dev][2] == smem)
-    S = cache_s[dev];
-  if (!S) {
-    S = 1;
-    for (int sc = std::min(8, nkb); sc >= 2 && S == 1; --sc) {
+  struct SKey {
+    int64_t v[4];
+  };
+  static PlanCache<SKey, int, 32> split_cache;
+  SKey key = {{dev, m_tiles, nkb, smem}};
+  int S = 1;
+  const bool ok = split_cache.get(key, S, [&](int& out) {
+    out = 1;
+    for (int sc = std::min(8, nkb); sc >= 2 && out == 1; --sc) {
       if (m_tiles * sc > sms) continue;
       cudaLaunchConfig_t qc = {};
       qc.gridDim = dim3(m_tiles * sc, 1, 1);
@@ -291,19 +274,17 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
       qc.attrs = &qa;
       qc.numAttrs = 1;
       int max_clusters = 0;
-      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, lowrank_down_kernel, &qc)) != cudaSuccess) return e;
-      if (m_tiles <= max_clusters) S = sc;
+      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, lowrank_down_kernel, &qc)) != cudaSuccess) return false;
+      if (m_tiles <= max_clusters) out = sc;
     }
-    if (dev < 64) {
-      cache_key[dev][0] = m_tiles;
-      cache_key[dev][1] = nkb;
-      cache_key[dev][2] = smem;
-      cache_s[dev] = S;
-    }
-  }
+    return true;
+  });
+  if (!ok) return e;
   CUtensorMap tX, tL1;
-  if (!tmap_bf16(&tX, X, (uint64_t)M, (uint64_t)K, BKL, BM) ||
-      !tmap_bf16(&tL1, L1, (uint64_t)K, (uint64_t)r, 64, BKL))
+  if (!make_tmap(&tX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)M, (uint64_t)K, BKL, BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L1, (uint64_t)K, (uint64_t)r, 64, BKL,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(m_tiles * S, 1, 1);
@@ -319,10 +300,15 @@ cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, in
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  LrParams prm{T, M, K, r, S, nst, err};
+  LrParams prm{T, M, K, r, S, nst, err, wait_ns, withhold};
   e = cudaLaunchKernelEx(&cfg, lowrank_down_kernel, prm, tX, tL1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_lowrank_down(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
+                                cudaStream_t st) {
+  return launch_lowrank_down_ex(X, L1, M, K, r, T, kWaitTimeoutNs, 0, st);
 }
 
 }  // namespace w4a4

@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "plan_cache.h"
 
 namespace w4a4 {
 
@@ -58,6 +59,10 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 constexpr int kStages = 2;  // 3 CTAs per SM each keep one block in flight
+
+struct RqShape {
+  int rows_per_blk, threads, smem, grid;
+};
 
 // Shared-memory stride of one staged group: g bf16 plus 16 bytes of padding,
 // so that the 16-byte reads of eight consecutive threads (eight consecutive
@@ -385,26 +390,21 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
 // costs the larger of a fixed memory latency and its bytes at HBM rate, and
 // the last wave costs as much as a full one.  (M = 4608, K = 3072, g = 128:
 // R = 5 gives 922 blocks on 444 CTAs -- three waves, the last 8% full;
-// R = 4 gives 1152 blocks on 592 CTAs -- two waves.)
-struct RqShape {
-  int rows_per_blk, threads, smem, grid;
-};
-
-template <int G, bool ROT, int QMAX, int MAXT, bool SR>
-cudaError_t pick_shape(int M, int K, int dev, RqShape& out) {
-  auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT, SR>;
+// R = 4 gives 1152 blocks on 592 CTAs -- two waves.)  A pure host function:
+// `per_sm(threads, smem)` gives the resident CTAs per SM of a candidate.
+template <class Occ>
+bool plan_rq_shape(int M, int K, int G, int maxt, int sms, Occ&& per_sm_of, RqShape& out) {
   const int gpr = K / G;
-  const int max_r = gpr >= MAXT ? 1 : MAXT / gpr;
-  int sms = 148;
-  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  const int max_r = gpr >= maxt ? 1 : maxt / gpr;
+  const int pitch = 2 * G + 16;   // group_stride<G>()
   double best = 1e30;
+  bool found = false;
   for (int r = max_r; r >= 1; --r) {
     const int threads = ((r * gpr + 31) / 32) * 32;
-    if (threads > MAXT) continue;
-    const int smem = kStages * r * gpr * group_stride<G>();
+    if (threads > maxt) continue;
+    const int smem = kStages * r * gpr * pitch;
     int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess) return e;
+    if (!per_sm_of(threads, smem, per_sm)) return false;
     per_sm = per_sm < 1 ? 1 : per_sm;
     const long nblk = (M + r - 1) / r;
     const long resident = (long)sms * per_sm;
@@ -415,9 +415,24 @@ cudaError_t pick_shape(int M, int K, int dev, RqShape& out) {
     if (cost < best * 0.999) {
       best = cost;
       out = RqShape{r, threads, smem, (int)grid};
+      found = true;
     }
   }
-  return cudaSuccess;
+  return found;
+}
+
+// Shapes already planned, keyed by (device, M, K, kernel instantiation).
+struct RqKey {
+  int64_t v[4];
+};
+PlanCache<RqKey, RqShape, 64>& rq_cache() {
+  static PlanCache<RqKey, RqShape, 64> c;
+  return c;
+}
+
+template <int G, bool ROT, int QMAX, int MAXT, bool SR>
+int64_t rq_kernel_id() {
+  return (int64_t)G | ((int64_t)ROT << 10) | ((int64_t)QMAX << 11) | ((int64_t)MAXT << 19) | ((int64_t)SR << 30);
 }
 
 template <int G, bool ROT, int QMAX, int MAXT, bool SR = false>
@@ -427,28 +442,23 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static int attr_set[64] = {0};
-  if (dev < 64 && !attr_set[dev]) {
+  static DeviceFlags attr_set;   // one per instantiation
+  if (!attr_set.done(dev)) {
     // the largest ring any shape uses (MAXT threads' groups, kStages deep)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStages * MAXT * group_stride<G>());
     if (e != cudaSuccess) return e;
-    attr_set[dev] = 1;
+    attr_set.set(dev);
   }
-  // shape of the last (M, K) seen on each device (deterministic, so a racing
-  // refresh only repeats the search)
-  static int cache_m[64] = {0}, cache_k[64] = {0};
-  static RqShape cache_shape[64];
   RqShape sh;
-  if (dev < 64 && cache_m[dev] == M && cache_k[dev] == K) {
-    sh = cache_shape[dev];
-  } else {
-    if ((e = pick_shape<G, ROT, QMAX, MAXT, SR>(M, K, dev, sh)) != cudaSuccess) return e;
-    if (dev < 64) {
-      cache_shape[dev] = sh;
-      cache_m[dev] = M;
-      cache_k[dev] = K;
-    }
-  }
+  const RqKey key = {{dev, M, K, rq_kernel_id<G, ROT, QMAX, MAXT, SR>()}};
+  const bool ok = rq_cache().get(key, sh, [&](RqShape& v) {
+    int sms = 0;
+    if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return false;
+    return plan_rq_shape(M, K, G, MAXT, sms, [&](int threads, int smem, int& per_sm) {
+      return (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) == cudaSuccess;
+    }, v);
+  });
+  if (!ok) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sh.grid, 1, 1);
   cfg.blockDim = dim3(sh.threads, 1, 1);
@@ -482,6 +492,31 @@ cudaError_t launch_rq_group(const uint16_t* X, int rows, int K, int group, uint8
 }
 
 }  // namespace
+
+// Launch-free planning of the rotate + quantize kernel's shape, for the
+// host-side thread-safety test: the same planner and cache type the launcher
+// uses, fed a fixed occupancy instead of a CUDA query.  `cached` selects a
+// shared eight-entry cache (constantly evicted when many shapes are asked
+// for) or a direct computation.
+bool plan_rotate_quantize_shape(int M, int K, int group, int sms, int resident_per_sm, bool cached, int out[4]) {
+  static PlanCache<RqKey, RqShape, 8> test_cache;
+  const int G = group == 64 ? 64 : 128;
+  const int maxt = K / G <= 128 ? 128 : 256;
+  auto make = [&](RqShape& v) {
+    return plan_rq_shape(M, K, G, maxt, sms, [&](int, int, int& per_sm) {
+      per_sm = resident_per_sm;
+      return true;
+    }, v);
+  };
+  RqShape sh;
+  const RqKey key = {{sms + 1000 * resident_per_sm, M, K, group}};
+  if (!(cached ? test_cache.get(key, sh, make) : make(sh))) return false;
+  out[0] = sh.rows_per_blk;
+  out[1] = sh.threads;
+  out[2] = sh.smem;
+  out[3] = sh.grid;
+  return true;
+}
 
 // Rows of X [rows, K] bf16 -> codes and one fp32 scale per row: packed
 // nibbles [rows, K/2] when qmax == 7 (symmetric) or qmax == 15 (asymmetric,
