@@ -144,12 +144,15 @@ w4a4_status w4a4_linear(const void* X, const uint8_t* Wq, const float* w_scale, 
  * running inside a runtime that forbids cudaMalloc after start-up -- and so
  * cannot pass the workspace w4a4_linear needs.
  *   Scratch: a fixed array of W4A4_NOALLOC_SCRATCH_BYTES inside the library,
- *     one per GPU that loads the library, kept until the process exits.  The
+ *     one per GPU that loads the library, held by that GPU's CUDA context for
+ *     as long as the context lives (normally until the process exits).  The
  *     call allocates nothing (no cudaMalloc, cudaFree or allocating library
  *     routine).  Layers whose w4a4_workspace_bytes(M, K, rank) exceeds the
  *     scratch are rejected with W4A4_ERR_WORKSPACE; use w4a4_linear for them.
- *   The first call on a device looks up the scratch address on that device
- *     (with it current); make that first call before any stream capture.
+ *   The first call in a context looks up the scratch address on that device
+ *     (with it current) and caches it per context, so a context recreated
+ *     after cudaDeviceReset looks it up again; make that first call before any
+ *     stream capture.
  *   All calls share the scratch.  Calls that may overlap on the GPU (other
  *     streams, other host threads) race on it and must be serialised by the
  *     caller.  The scratch keeps the last call's contents; every byte a call

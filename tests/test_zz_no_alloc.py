@@ -35,9 +35,14 @@ def test_noalloc_matches_linear_on_two_calls_in_a_row():
     build.build()
     w4.load_library()
     results = []
-    # two different layers back to back: the second call reuses the scratch
-    # the first one left behind
-    for seed, (M, K, N, g, r) in [(11, (640, 3072, 1024, 128, 0)), (12, (200, 1280, 520, 64, 32))]:
+    # layers back to back on the shared scratch, each checked against
+    # w4a4_linear: a large one that fills most of the scratch, a smaller one
+    # whose codes, scales and T sit at other offsets over that data, then one
+    # larger than the second with yet another geometry, so every region a call
+    # reads was last written by a different layer (stale bytes would show)
+    layers = [(10, (1536, 3072, 1024, 128, 64)), (11, (640, 3072, 1024, 128, 0)),
+              (12, (200, 1280, 520, 64, 32)), (13, (1000, 2048, 264, 64, 48))]
+    for seed, (M, K, N, g, r) in layers:
         X, W, L1, L2, b = _layer(seed, M, K, N, g, r)
         Wq, ws = w4.w4a4_quantize_weights(W, g)
         ref = w4.w4a4_linear(X, Wq, ws, g, L1, L2, b)

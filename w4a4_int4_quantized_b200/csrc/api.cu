@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "plan_cache.h"
 #include "w4a4.h"
 
 namespace w4a4 {
@@ -15,7 +16,6 @@ __device__ unsigned int g_device_error_word = 0u;
 namespace {
 
 constexpr int kMaxDevices = 64;
-std::atomic<unsigned int*> g_err_ptr[kMaxDevices];
 std::atomic<int> g_dev_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -63,16 +63,12 @@ size_t round256(size_t x) { return (x + 255u) & ~size_t(255u); }
 }  // namespace
 
 unsigned int* device_error_word() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  unsigned int* p = g_err_ptr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_device_error_word) != cudaSuccess) return nullptr;
-    p = static_cast<unsigned int*>(addr);
-    g_err_ptr[dev].store(p, std::memory_order_release);
+  void* addr = nullptr;
+  if (symbol_address_cached(reinterpret_cast<const void*>(&g_device_error_word), &addr) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return p;
+  return static_cast<unsigned int*>(addr);
 }
 
 }  // namespace w4a4

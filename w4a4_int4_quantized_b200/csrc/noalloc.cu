@@ -11,6 +11,7 @@
 #include <atomic>
 #include <cstdint>
 
+#include "plan_cache.h"
 #include "w4a4.h"
 
 namespace w4a4 {
@@ -23,29 +24,18 @@ static_assert(kScratchBytes % 256 == 0, "scratch size");
 // device address comes from cudaGetSymbolAddress below.
 __device__ __align__(256) uint8_t g_linear_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::atomic<uint8_t*> g_scratch_addr[kMaxDevices];
-
-// Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// Device address of the scratch in the current context, looked up with
+// cudaGetSymbolAddress (with that device current) the first time a context
+// asks and cached per context, so a context recreated after cudaDeviceReset
+// looks the address up again.
 w4a4_status scratch_for_current_device(uint8_t** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  void* addr = nullptr;
+  if (symbol_address_cached(reinterpret_cast<const void*>(&g_linear_scratch), &addr) != cudaSuccess ||
+      addr == nullptr) {
     cudaGetLastError();
     return W4A4_ERR_CUDA;
   }
-  if (dev < 0 || dev >= kMaxDevices) return W4A4_ERR_UNSUPPORTED_DEVICE;
-  uint8_t* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_linear_scratch) != cudaSuccess || addr == nullptr) {
-      cudaGetLastError();
-      return W4A4_ERR_CUDA;
-    }
-    p = static_cast<uint8_t*>(addr);
-    g_scratch_addr[dev].store(p, std::memory_order_release);
-  }
-  *out = p;
+  *out = static_cast<uint8_t*>(addr);
   return W4A4_OK;
 }
 

@@ -87,6 +87,16 @@ struct DeviceFlags {
   }
 };
 
+// Unique id of the calling thread's current CUDA context (0 when there is
+// none or the driver cannot say).  Device addresses of module globals are
+// cached per context id, so a context recreated after cudaDeviceReset gets
+// its own lookup instead of a stale address.
+unsigned long long current_context_id();
+
+// Device address of a module global (__device__ variable) in the current
+// context, looked up once per context.
+cudaError_t symbol_address_cached(const void* symbol, void** out);
+
 // Number of SMs of a device, looked up once per device.
 inline cudaError_t device_sm_count(int dev, int* out) {
   static std::atomic<int> cached[64];

@@ -7,6 +7,8 @@
 #include <cudaTypedefs.h>
 #include <string.h>
 
+#include <utility>
+
 #include "plan_cache.h"
 #include "tmap.h"
 
@@ -73,6 +75,56 @@ bool make_tmap(CUtensorMap* out, CUtensorMapDataType dt, int esize, const void* 
   const uint64_t strides[1] = {cols * (uint64_t)esize};
   const uint32_t box[2] = {box_cols, box_rows};
   return make_tmap_nd(out, dt, esize, base, 2, dims, strides, box, swz);
+}
+
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static const std::pair<GetCurrent, GetId> fns = [] {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess)
+      f1 = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      f2 = nullptr;
+    return std::make_pair(reinterpret_cast<GetCurrent>(f1), reinterpret_cast<GetId>(f2));
+  }();
+  if (!fns.first || !fns.second) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (fns.first(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (fns.second(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+cudaError_t symbol_address_cached(const void* symbol, void** out) {
+  struct Key {
+    int64_t v[2];
+  };
+  struct Val {
+    void* p;
+  };
+  static PlanCache<Key, Val, 64> cache;
+  unsigned long long ctx = current_context_id();
+  Val v{nullptr};
+  if (ctx != 0) {
+    const Key key = {{(int64_t)ctx, (int64_t)reinterpret_cast<uintptr_t>(symbol)}};
+    if (cache.find(key, v)) {
+      *out = v.p;
+      return cudaSuccess;
+    }
+  }
+  // the lookup also makes the device's primary context current if the
+  // calling thread had none yet; the id is taken again afterwards
+  const cudaError_t e = cudaGetSymbolAddress(&v.p, symbol);
+  if (e != cudaSuccess) return e;
+  ctx = current_context_id();
+  if (ctx != 0) cache.insert(Key{{(int64_t)ctx, (int64_t)reinterpret_cast<uintptr_t>(symbol)}}, v);
+  *out = v.p;
+  return cudaSuccess;
 }
 
 }  // namespace w4a4
