@@ -59,6 +59,7 @@ def _load():
         lib.oracle_f32_to_bf16.argtypes = [P, L, P]
         lib.oracle_f64_to_bf16.argtypes = [P, L, P]
         lib.oracle_lora_merge.argtypes = [P, P, I, P, P, I, ctypes.c_float, I, I, P, P]
+        lib.oracle_lowrank_up.argtypes = [P, P, L, L, I, ctypes.c_double, P]
         lib.oracle_gelu_tanh.argtypes = [P, L, P]
         lib.oracle_philox4x64.argtypes = [P, P, P]
         lib.oracle_sr_uniform.argtypes = [L, ctypes.c_uint64, P]
@@ -339,10 +340,21 @@ def linear_w4a4_lora(X, W, g, L1, L2, A, B, scale: float, bias=None):
     fp64 from the bf16 operands (unmerged)."""
     base = linear_w4a4(X, W, g, L1, L2, bias)
     TA = lowrank_down(X, A)
-    lora = float(np.float32(scale)) * (TA @ bf16_to_f64(B))
     out = dict(base)
-    out["Y"] = base["Y"] + lora
+    out["Y"] = lowrank_up(TA, B, float(np.float32(scale)), base["Y"])
     out["T_lora"] = TA
+    return out
+
+
+def lowrank_up(T, U, scale: float, Y):
+    """Y + scale * (T U) in fp64 (oracle_lowrank_up): T fp64 [M, r], U bf16
+    bits [r, N], Y fp64 [M, N]; returns a new array."""
+    T = np.ascontiguousarray(T, dtype=np.float64)
+    U = _bf16(U)
+    M, r = T.shape
+    N = U.shape[1]
+    out = np.array(Y, dtype=np.float64, order="C", copy=True)
+    _load().oracle_lowrank_up(_ptr(T), _ptr(U), M, N, r, float(scale), _ptr(out))
     return out
 
 

@@ -405,6 +405,19 @@ void oracle_lora_merge(const uint16_t *L1, const uint16_t *L2, int r, const uint
 /* Y[m][n] = ((acc * sa[m]) * sw[n]) * (1/g) + sum_j T[m][j] * L2[j][n] + bias[n]
    in fp64.  g == 0 means no rotation (factor 1).  T/L2 are ignored when r == 0;
    bias may be NULL. */
+/* Y[m][n] += scale * sum_j T[m][j] * U[j][n] in fp64, j in index order: the
+ * up-projection of a low-rank branch applied on its own (the runtime LoRA
+ * beside the SVDQuant branch, unmerged).  T fp64 [M, r], U bf16 [r, N]. */
+void oracle_lowrank_up(const double *T, const uint16_t *U, long M, long N, int r, double scale, double *Y) {
+    #pragma omp parallel for schedule(static)
+    for (long m = 0; m < M; ++m)
+        for (long n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int j = 0; j < r; ++j) acc += T[m * r + j] * (double)bf16_to_f32(U[(long)j * N + n]);
+            Y[m * N + n] += scale * acc;
+        }
+}
+
 void oracle_epilogue(const int32_t *acc, const float *sa, const float *sw, long M, long N, int g,
                      const double *T, const uint16_t *L2, int r, const uint16_t *bias, double *Y) {
     const double inv_g = (g > 0) ? 1.0 / (double)g : 1.0;

@@ -623,3 +623,22 @@ def test_lora_bake_bound_and_identities():
     out = oracle.bake_requantize(W, A, B, 0.75, 64, seed=9)
     assert np.array_equal(out["w_baked"], Wb)
     assert np.all(np.abs(out["w_q"]) <= 8)
+
+
+def test_lowrank_up_is_the_fp64_product():
+    """oracle_lowrank_up adds scale * (T U) in fp64: pinned against NumPy's
+    matmul; a transposed or unscaled operand does not match."""
+    rng = np.random.default_rng(77)
+    M, r, N = 9, 32, 40
+    T = rng.standard_normal((M, r))
+    U = _bf16(rng.standard_normal((r, N), dtype=np.float32))
+    Y0 = rng.standard_normal((M, N))
+    got = oracle.lowrank_up(T, U, 0.375, Y0)
+    ref = Y0 + 0.375 * (T @ oracle.bf16_to_f64(U))
+    assert np.allclose(got, ref, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(oracle.lowrank_up(T, U, 0.0, Y0), Y0)
+    assert not np.allclose(got, Y0 + (T @ oracle.bf16_to_f64(U)), rtol=1e-6)
+    Usq = _bf16(rng.standard_normal((r, r), dtype=np.float32))
+    Tsq = rng.standard_normal((r, r))
+    assert not np.allclose(oracle.lowrank_up(Tsq, Usq, 1.0, np.zeros((r, r))),
+                           Tsq @ oracle.bf16_to_f64(Usq).T, rtol=1e-6)
