@@ -36,6 +36,16 @@ sys.path.insert(0, ROOT)
 
 INT8_NOMINAL_TOPS = 4500.0     # B200 dense INT8 tensor peak (datasheet)
 HBM_NOMINAL_GBS = 8000.0
+# measured on this part: one pair MMA M256 N256 K32 int8 every 128 cycles
+# = 8192 int8 MAC per clock per SM; the clock-adjusted peak uses it with the
+# SM clock sampled during the run
+INT8_MAC_PER_CLK_PER_SM = 8192
+
+
+def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
+    if not sm_mhz:
+        return None
+    return 2.0 * INT8_MAC_PER_CLK_PER_SM * sms * sm_mhz * 1e6 / 1e12
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # the ncu captures summarised in profiles/, valid only for the kernel source
@@ -423,6 +433,110 @@ def run_block(args):
         "gpu_launches": sum(2 if L["spec"].w8a8 else 3 for L in layers) * args.steps, "clocks": clk}), flush=True)
 
 
+def run_sweep(args):
+    """Shape sweep (one GPU): M in {256, 1024, 4608, 9216, 16384} x (K, N) in
+    {(3072, 3072), (3072, 9216), (3072, 12288), (12288, 3072)} x rank in
+    {0, 16, 64, 128} for W4A4 (group 128), plus the W4A8 layer at every
+    (M, K, N), and the tiny single layer (M=64, K=N=256, group 64, rank 16).
+    Inputs: X ~ N(0,1) with 1% of channels x100, W ~ N(0, 0.02), L1, L2 ~
+    N(0, 0.01), bias ~ N(0, 0.01), drawn on the device from fixed seeds.  Each
+    point: the whole-layer call (w4a4_linear / w4a8_linear), L2 flushed before
+    every timed call (a 256 MB write outside the events), CUDA events around
+    the call, median over --steps calls.  One JSON line per point."""
+    import torch
+    import w4a4_int4_quantized_b200 as w4
+    w4.load_library()
+    torch.cuda.set_device(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    pk = _peaks()
+    i8 = 2.0 * pk["bf16"]
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = time.perf_counter()
+
+    def draw(shape, seed, std):
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed)
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+    def acts(M, K, seed):
+        X = torch.randn((M, K), generator=torch.Generator(device="cuda").manual_seed(seed), device="cuda")
+        ch = torch.randperm(K, generator=torch.Generator(device="cuda").manual_seed(seed + 1), device="cuda")
+        X[:, ch[: max(1, round(0.01 * K))]] *= 100.0
+        return X.to(torch.bfloat16)
+
+    def timed(fn):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            ev[0].record(stream)
+            fn()
+            ev[1].record(stream)
+            ev[1].synchronize()
+            ts.append(ev[0].elapsed_time(ev[1]) * 1e3)
+        return statistics.median(ts)
+
+    def emit(name, M, K, N, g, r, variant, us, code_bytes):
+        ops = 2.0 * M * N * K
+        lr = 2.0 * M * r * (K + N)
+        wbytes = N * K // 2 if variant != "w8a8" else N * K
+        bytes_ = M * K * 2 + M * N * 2 + wbytes + (M * r * 2 * 2 + (K + N) * r * 2 if r else 0) + code_bytes
+        roof_us = max((ops / (4500e12) + lr / (2250e12)) * 1e6, bytes_ / (pk["hbm_gbs"] * 1e9) * 1e6)
+        print(json.dumps({"sweep": name, "variant": variant, "M": M, "K": K, "N": N, "group": g, "rank": r,
+                          "us": us, "tops": ops / (us * 1e-6) / 1e12,
+                          "frac_of_int8_nominal": ops / (us * 1e-6) / 1e12 / INT8_NOMINAL_TOPS,
+                          "frac_of_int8_measured": ops / (us * 1e-6) / 1e12 / i8,
+                          "roofline_us": roof_us, "frac_of_roofline": roof_us / us,
+                          "l2": "flushed before every call"}), flush=True)
+
+    # the tiny single layer
+    X = acts(64, 256, 0)
+    Wq, ws = w4.w4a4_quantize_weights(draw((256, 256), 1, 0.02), 64)
+    L1, L2 = draw((256, 16), 2, 0.01), draw((16, 256), 3, 0.01)
+    ws_buf = torch.empty((w4.w4a4_workspace_bytes(64, 256, 16),), dtype=torch.uint8, device="cuda")
+    Y = torch.empty((64, 256), dtype=torch.bfloat16, device="cuda")
+    us = timed(lambda: w4.w4a4_linear(X, Wq, ws, 64, L1, L2, None, Y=Y, workspace=ws_buf))
+    emit("tiny", 64, 256, 256, 64, 16, "w4a4", us, 64 * 128)
+
+    Ms = [256, 1024, 4608, 9216, 16384]
+    KN = [(3072, 3072), (3072, 9216), (3072, 12288), (12288, 3072)]
+    ranks = [0, 16, 64, 128]
+    for ki, (K, N) in enumerate(KN):
+        seed = 1000 + 10 * ki
+        W = draw((N, K), seed, 0.02)
+        Wq, ws = w4.w4a4_quantize_weights(W, 128)
+        Wq8, ws8, wz8 = w4.w4a8_quantize_weights(W, 128)
+        b = draw((N,), seed + 1, 0.01)
+        L1f, L2f = draw((K, 128), seed + 2, 0.01), draw((128, N), seed + 3, 0.01)
+        del W
+        for M in Ms:
+            X = acts(M, K, seed + 5 + M)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            for r in ranks:
+                L1 = L1f[:, :r].contiguous() if r else None
+                L2 = L2f[:r].contiguous() if r else None
+                wsb = torch.empty((w4.w4a4_workspace_bytes(M, K, r),), dtype=torch.uint8, device="cuda")
+                us = timed(lambda: w4.w4a4_linear(X, Wq, ws, 128, L1, L2, b, Y=Y, workspace=wsb))
+                emit("c5", M, K, N, 128, r, "w4a4", us, M * K // 2)
+                del wsb
+            wsb = torch.empty((w4.w4a8_workspace_bytes(M, K),), dtype=torch.uint8, device="cuda")
+            us = timed(lambda: w4.w4a8_linear(X, Wq8, ws8, wz8, 128, b, Y=Y, workspace=wsb))
+            emit("c5", M, K, N, 128, 0, "w4a8", us, M * K)
+            del X, Y, wsb
+            torch.cuda.empty_cache()
+    clocks.mark(t0, time.perf_counter())
+    clk = clocks.stop()
+    err = w4.w4a4_get_device_error()
+    if err:
+        raise SystemExit(f"device error word {err:#x}")
+    print(json.dumps({"sweep": "done", "clocks": clk, "peaks": pk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -433,6 +547,10 @@ def main():
     ap.add_argument("--sets", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--soak-ms", type=float, default=400.0,
+                    help="run blocks of --steps steps for this long before the timed region (clock record)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="shape sweep: M x (K, N) x rank for W4A4 plus the W4A8 points, one JSON line each")
     ap.add_argument("--block", action="store_true",
                     help="time the linear layers of the double-stream block at batch 2 (M=9216)")
     ap.add_argument("--bake-lora", type=int, default=0,
@@ -448,6 +566,12 @@ def main():
         raise SystemExit("--warmup must be >= 3")
 
     from w4a4_int4_quantized_b200 import inputs
+    if args.sweep:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the sweep is measured by the GPU arm only"}))
+            return
+        run_sweep(args)
+        return
     if args.block:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the block is measured by the GPU arm only"}))
@@ -545,17 +669,41 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # clock soak: blocks of K steps back to back for --soak-ms (untimed for
+    # `value`; each block timed on its own for the `sustained` figure), so the
+    # clock record sampled across soak + timed region covers the clock the
+    # timed steps ran at, however short they are
+    e_blk = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    soak_ms, soak_blocks = [], 0
+    wall0 = time.perf_counter()
+    while args.soak_ms > 0 and (time.perf_counter() - wall0) * 1e3 < args.soak_ms:
+        e_blk[0].record(stream)
+        for i in range(args.steps):
+            step(sets[i % len(sets)])
+        e_blk[1].record(stream)
+        e_blk[1].synchronize()
+        soak_ms.append(e_blk[0].elapsed_time(e_blk[1]) / args.steps)
+        soak_blocks += 1
+    if world > 1:
+        # every rank takes the same collective steps: agree on the block count
+        nb = torch.tensor([soak_blocks], device="cuda")
+        dist.all_reduce(nb, op=dist.ReduceOp.MAX)
+        for _ in range(int(nb.item()) - soak_blocks):
+            for i in range(args.steps):
+                step(sets[i % len(sets)])
+        torch.cuda.synchronize()
+        dist.barrier()
     # timed region: K whole layers back to back (no events between kernels,
     # so each launch may overlap the previous kernel's tail)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    wall0 = time.perf_counter()
+    t_timed = time.perf_counter()
     e_start.record(stream)
     for i in range(args.steps):
         step(sets[i % len(sets)])
     e_end.record(stream)
     torch.cuda.synchronize()
-    wall = time.perf_counter() - wall0
-    clocks.mark(wall0, wall0 + wall)
+    wall = time.perf_counter() - t_timed
+    clocks.mark(wall0, t_timed + wall)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -616,8 +764,26 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         te = max_over_ranks(e0.elapsed_time(e1), device="cuda")
+        # the same step with events between its three parts (for the split)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        parts = [0.0, 0.0, 0.0]
+        for _ in range(args.e2e_steps):
+            ev[0].record(stream)
+            s["X"].copy_(hx, non_blocking=True)
+            ev[1].record(stream)
+            linear()
+            ev[2].record(stream)
+            hy.copy_(s["Y"], non_blocking=True)
+            ev[3].record(stream)
+            torch.cuda.synchronize()
+            for j in range(3):
+                parts[j] += ev[j].elapsed_time(ev[j + 1])
         e2e = {"value": ops * args.e2e_steps * world / (te * 1e-3) / 1e12, "unit": "TOPS",
-               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2}
+               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+               "us_per_step": te / args.e2e_steps * 1e3,
+               "split_us": {"h2d": parts[0] / args.e2e_steps * 1e3, "layer": parts[1] / args.e2e_steps * 1e3,
+                            "d2h": parts[2] / args.e2e_steps * 1e3,
+                            "note": "pinned host copies over PCIe around one w4a4_linear call"}}
 
     if rank == 0:
         pk = _peaks()
@@ -628,21 +794,33 @@ def main():
         # the burst bf16 figure x the nominal int8 : bf16 ratio of 2
         int8_peak = 2.0 * pk["bf16"]
         k1_bytes = M * K * 2 + (M * K if w4a8 else M * K // 2) + M * 4
+        adj = clock_adjusted_peak_tops(clk.get("sm_mhz"))
         line = {
             "metric": _metric_name(args.variant, spec),
             "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "us_per_layer": total_ms / args.steps * 1e3,
             "frac_of_int8_nominal_peak": value / INT8_NOMINAL_TOPS,
+            "layer_frac": {"of_int8_nominal": value / INT8_NOMINAL_TOPS,
+                           "of_int8_measured": value / world / (2.0 * pk["bf16"]),
+                           "of_int8_clock_adjusted": (value / world / adj) if adj else None,
+                           "clock_adjusted_peak_tops": adj,
+                           "note": "whole layer (K1 + K2) per GPU; clock-adjusted = 8192 int8 MAC/clk/SM x 2 x "
+                                   "148 SMs x median sampled SM clock"},
+            "sustained": {"us_per_layer_median": statistics.median(soak_ms) * 1e3 if soak_ms else None,
+                          "blocks": len(soak_ms), "steps_per_block": args.steps,
+                          "note": "blocks of K steps run back to back before the timed region (clock soak)"},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": ("int8 activations x 4-bit zero-pointed weights" if w4a8 else "int4 codes")
                      + " (int8 MMA, int32 acc), bf16 in/out", "data": "synthetic",
             "config": {"workload": spec.name, "variant": args.variant, "M": M, "K": K, "N": N, "group": g, "rank": r,
                        "lora_rank": args.lora,
                        "bias": spec.bias, "parallelism": f"replicas x{world} (token shards, no exchange)",
-                       "l2": f"{args.sets} rotating input sets (> L2)"},
+                       "l2": f"{args.sets} rotating input sets (> L2)",
+                       "clock_soak_ms": args.soak_ms},
             "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3, "note": "each kernel timed alone, back to back"},
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
                          "frac": k2_tops / int8_peak,
+                         "frac_clock_adjusted": (k2_tops / adj) if adj else None,
                          "traffic": _traffic("gemm_w4a8" if w4a8 else "gemm", spec.name),
                          "peak_note": f"int8 = 2 x {pk['source']} burst bf16 {pk['bf16']} TFLOP/s (kernel timed "
                                       f"alone); {2.0 * pk['bf16_sustained']:.0f} with the sustained figure"},

@@ -28,3 +28,18 @@ def pytest_collection_modifyitems(config, items):
         for item in items:
             if "gpu" in item.keywords:
                 item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _device_error_word_stays_clear(request):
+    """After every GPU test, the library's device error word must be clear:
+    a bounded wait that ran out inside any kernel fails the test that ran it
+    (the wait-timeout self-test clears the word itself)."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    import w4a4_int4_quantized_b200 as w4
+    if w4._lib is None:
+        return
+    code = w4.w4a4_get_device_error()
+    assert code == 0, f"device error word {code:#x} after {request.node.name}"

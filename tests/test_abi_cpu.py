@@ -251,7 +251,7 @@ def test_launch_plan_cache_under_host_threads(lib):
     shapes = [(m, k, g) for m in (1, 2, 37, 256, 1000, 4608, 9216, 16384)
               for k in (256, 3072, 12288) for g in (64, 128)]
     expect = {sh: w4.w4a4_plan_rotate_quantize(*sh, cached=False) for sh in shapes}
-    assert expect[(4608, 3072, 128)] == (4, 96, 4 * 24 * 272 * 2, 592)
+    assert expect[(4608, 3072, 128)] == (4, 96, 2 * 4 * 3072 * 2 + 1024, 592)
 
     def worker(seed):
         rnd = random.Random(seed)

@@ -89,26 +89,29 @@ constexpr int kBarBytes = 512;
 
 // MODE 0: W8A8 (int8 x int8, TMA straight into the MMA layout); 1: W4A4
 // (packed INT4 x packed INT4, both widened, A into TMEM); 2: W4A8 (the int8
-// activation tile is read by the MMA straight from its TMA stage; packed
-// unsigned 4-bit weights are widened with their zero point subtracted).
+// activation tile is read by the MMA straight from its own TMA ring, freed by
+// the MMA commit; packed unsigned 4-bit weights are widened with their zero
+// point subtracted and their packed stages are freed by the widen warps).
 template <int MODE, bool LR>
 struct Cfg {
   static constexpr bool PACKED = MODE != 0;          // the widen pipeline runs
-  static constexpr int PS = 4;                      // TMA stages (A + packed B), kSets apart
+  static constexpr int PS = 4;                      // packed TMA stages (W4A4: A + B; W4A8: B), kSets apart
   static constexpr int US = MODE == 2 ? 4 : (LR ? 5 : 7);  // widened stages (W4A8: B only)
+  static constexpr int AS = MODE == 2 ? 5 : 0;       // W4A8: int8 A stages, read by the MMA in place
   static constexpr int kLead = US - 2;               // k-blocks widened ahead of an epilogue
   static constexpr int BN = 256;                     // N per pair tile
   static constexpr int BNH = BN / 2;                 // B rows staged per CTA
   static constexpr int kARow = MODE == 2 ? BK : BK / 2;  // bytes of an A row per k-block
-  static constexpr int kPkA = BM * kARow;            // A stage (8 KB packed, 16 KB int8)
+  static constexpr int kPkA = MODE == 1 ? BM * kARow : 0;  // packed A in the packed stage (W4A4 only)
   static constexpr int kPkB = BNH * BK / 2;
   static constexpr int kPkStage = kPkA + kPkB;
   static constexpr int kWideB = BNH * BK;            // widened B stage
   static constexpr int kI8A = BM * BK;               // INT8 stages
   static constexpr int kI8B = BNH * BK;
   static constexpr int kI8Stage = kI8A + kI8B;
-  static constexpr int kRing = PACKED ? PS * kPkStage + US * kWideB : S8 * kI8Stage;
+  static constexpr int kRing = PACKED ? PS * kPkStage + US * kWideB + AS * kI8A : S8 * kI8Stage;
   static constexpr int kWOff = PS * kPkStage;        // widened B ring
+  static constexpr int kAOff = kWOff + US * kWideB;  // W4A8 int8 A ring
   static constexpr int kLrT = BM * LRC * 2;          // T chunk: 128 rows x 128 ranks, two 64-wide boxes
   static constexpr int kLrL2 = BNH * LRC * 2;        // L2 chunk: 128 ranks x BNH columns, two 64-wide boxes
   static constexpr int kLrBytes = LR ? kLrT + kLrL2 : 0;
@@ -130,7 +133,7 @@ struct Cfg {
   // order, so a phase-parity wait can never match a fill two phases old
   static_assert(PS % kSets == 0, "each widen set owns its packed stages");
   static_assert(US >= kSets && kLead >= 1, "widened ring");
-  static_assert(kWOff % 1024 == 0, "128-byte swizzle atoms");
+  static_assert(kWOff % 1024 == 0 && kAOff % 1024 == 0, "128-byte swizzle atoms");
   static_assert(!LR || MODE == 1, "low-rank branch: W4A4 only");
   static_assert(!LR || kOutStageBytes <= kLrBytes, "epilogue staging inside the low-rank buffer");
 };
@@ -153,6 +156,8 @@ struct Barriers {
   uint64_t lr_free;      // the epilogue's stores staged in the low-rank buffer have been read
   uint64_t acc_full;
   uint64_t acc_empty;    // even CTA: both CTAs' epilogues have read the accumulators
+  uint64_t a_full[8];    // W4A8: this CTA's int8 A stage landed (TMA)
+  uint64_t a_empty[8];   // W4A8: the MMAs reading an A stage completed
   uint64_t drain;
   uint32_t tmem_base;
 };
@@ -269,10 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int s = 0; s < 8; ++s) {
         mbar_init(&bar->tma_full[s], 1);
-        // W4A4: the 4 widen warps of a set read the stage; W4A8: the same 4
-        // warps plus the MMA commit (the MMA reads A from the stage); W8A8:
-        // the MMA commit
-        mbar_init(&bar->tma_empty[s], MODE == 1 ? kSetWarps : (MODE == 2 ? kSetWarps + 1 : 1));
+        // packed modes: the 4 widen warps of a set read the stage; W8A8: the
+        // MMA commit
+        mbar_init(&bar->tma_empty[s], PACKED ? kSetWarps : 1);
+        mbar_init(&bar->a_full[s], 1);
+        mbar_init(&bar->a_empty[s], 1);
         mbar_init(&bar->full[s], PACKED ? 2 * kSetWarps : 1);  // a set's warps in both CTAs, or 1 relay
         mbar_init(&bar->empty[s], 1);
       }
@@ -305,6 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int NS = PACKED ? PS : S8;
       constexpr int kStageBytes = PACKED ? C::kPkStage : C::kI8Stage;
       constexpr int kABytes = PACKED ? C::kPkA : C::kI8A;
+      int as = 0;            // W4A8: A ring slot and phase
+      uint32_t a_ph = 0;
       constexpr int kColA = PACKED ? C::kARow : BK;   // bytes per k-block of an A / B row
       constexpr int kColB = PACKED ? BK / 2 : BK;
       int s = 0;
@@ -365,9 +373,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
           mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
-          tma_load_2d(dst, &tmA, kb * kColA, row_a, &bar->tma_full[s]);
+          if (MODE != 2) tma_load_2d(dst, &tmA, kb * kColA, row_a, &bar->tma_full[s]);
           tma_load_2d(dst + kABytes, &tmB, kb * kColB, row_b, &bar->tma_full[s]);
           if (++s == NS) { s = 0; ph ^= 1u; }
+          if constexpr (MODE == 2) {
+            // the int8 A tile into its own ring, once the MMAs have freed the slot
+            if (!mbar_wait(&bar->a_empty[as], a_ph ^ 1u)) {
+              set_device_error(prm.err, kDevErrTimeoutEmpty);
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bar->a_full[as], (uint32_t)C::kI8A);
+            tma_load_2d(sbase + (uint32_t)(C::kAOff + as * C::kI8A), &tmA, kb * BK, row_a, &bar->a_full[as]);
+            if (++as == C::AS) { as = 0; a_ph ^= 1u; }
+          }
           if (LR && kb == nk / 2) lr_eligible = (i + 1) * lr_chunks;
         }
       }
@@ -418,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_i8(2 * BM, BN);
       constexpr uint32_t idesc_lr = idesc_bf16(2 * BM, BN, false, true);
       constexpr int NS = PACKED ? US : S8;
-      int s = 0, ps = 0;   // widened / TMA stage of the k-block
+      int s = 0, ps = 0;   // widened stage / TMA stage of the k-block (W4A8: A ring slot)
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
         for (int kb = 0; kb < nk; ++kb) {
@@ -437,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (kb | ks) != 0 ? 1u : 0u);
               tc_commit_pair_mc(&bar->empty[s], 0x3);
             } else if (MODE == 2) {
-              const uint32_t a_stage = sbase + (uint32_t)(ps * C::kPkStage);
+              const uint32_t a_stage = sbase + (uint32_t)(C::kAOff + ps * C::kI8A);
               const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
 #pragma unroll
               for (int ks = 0; ks < BK / 32; ++ks)
@@ -445,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
                                (kb | ks) != 0 ? 1u : 0u);
               tc_commit_pair_mc(&bar->empty[s], 0x3);
-              tc_commit_pair_mc(&bar->tma_empty[ps], 0x3);
+              tc_commit_pair_mc(&bar->a_empty[ps], 0x3);
             } else {
               const uint32_t a_stage = sbase + (uint32_t)(s * C::kI8Stage);
 #pragma unroll
@@ -458,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (++s == NS) s = 0;
-          if (++ps == PS) ps = 0;
+          if (++ps == (MODE == 2 ? C::AS : PS)) ps = 0;
         }
         // the integer product of the tile is complete
         if (ok && lane == 0) tc_commit_pair_mc(&bar->acc_full, 0x3);
@@ -626,6 +645,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kWidenA) {
         tmem_wait_st();
         tc_fence_before();
+      }
+      if constexpr (MODE == 2) {
+        // the k-block also needs this CTA's int8 A tile: the hand-off below
+        // then tells the issuer that A and B have landed in this CTA
+        if (!mbar_wait(&bar->a_full[g % C::AS], (uint32_t)(g / C::AS) & 1u)) {
+          set_device_error(prm.err, kDevErrTimeoutFull);
+          return false;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);

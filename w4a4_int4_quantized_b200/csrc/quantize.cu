@@ -19,11 +19,16 @@
 // with exact division.  Each thread writes its codes as 16-byte stores.
 #include <cuda_bf16.h>
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "plan_cache.h"
+#include "tmap.h"
 
 namespace w4a4 {
+
+unsigned int* device_error_word();
 
 namespace {
 
@@ -49,26 +54,11 @@ __device__ __forceinline__ uint32_t pack_bytes4(uint32_t t0, uint32_t t1, uint32
   return __byte_perm(__byte_perm(t0, t1, 0x0040), __byte_perm(t2, t3, 0x0040), 0x5410);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-constexpr int kStages = 2;  // 3 CTAs per SM each keep one block in flight
+constexpr int kStages = 2;  // stages (blocks of rows) per CTA, both requested up front
 
 struct RqShape {
   int rows_per_blk, threads, smem, grid;
 };
-
-// Shared-memory stride of one staged group: g bf16 plus 16 bytes of padding,
-// so that the 16-byte reads of eight consecutive threads (eight consecutive
-// groups) fall in eight different bank groups.
-template <int G>
-constexpr int group_stride() { return G * 2 + 16; }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -117,11 +107,6 @@ __device__ __forceinline__ void quantize_block8(const float2* P8, float2 ih, flo
   }
 }
 
-// Persistent CTAs walk blocks of R consecutive rows.  Blocks are staged in a
-// 3-deep shared-memory ring with cp.async (coalesced 16-byte copies, no
-// registers held while in flight), so the loads of the next blocks overlap
-// the rotation and quantization of the current one.  One thread owns one
-// group; its g values go from shared memory straight into float2 registers.
 // Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
 // easy as 1, 2, 3", SC 2011): 10 rounds of two 64 x 64 -> 128-bit products
 // on a 4-word counter with a Weyl-sequence key schedule.
@@ -186,6 +171,17 @@ __device__ __forceinline__ float fkey_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// Persistent CTAs walk blocks of R consecutive rows.  Each block arrives in
+// a shared-memory stage by TMA: X viewed as [rows * K/g groups][g/64 halves]
+// [64 elements], one box per half covering the block's R * K/g groups, with
+// the 128-byte swizzle, so the 16-byte reads of eight consecutive threads
+// (eight consecutive groups) hit eight different bank groups.  Both stages
+// are requested at once when the kernel starts and each is refilled as soon
+// as every thread has taken its group out of it, so the HBM stream runs
+// while the rows already delivered are rotated and quantized.  One thread
+// owns one group; its g values go from shared memory straight into float2
+// registers.
+//
 // QMAX: 7 = symmetric INT4 (packed), 127 = symmetric INT8, 15 = asymmetric
 // 4-bit with a zero point (W4A8 weights, packed unsigned codes): per row
 // s = fl32(fl32(max - min) / 15), z = clamp(rint(fl32(-min / s)), 0, 15),
@@ -194,80 +190,99 @@ __device__ __forceinline__ float fkey_value(uint32_t k) {
 // instead of round-to-nearest (re-quantizing weights with a baked LoRA).
 template <int G, bool ROT, int QMAX, int MAXT, bool SR = false>
 __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
-    rotate_quantize_kernel(const uint16_t* __restrict__ X, int M, int K, int rows_per_blk, uint8_t* __restrict__ out,
-                           float* __restrict__ scale, uint8_t* __restrict__ zero, unsigned long long seed) {
+    rotate_quantize_kernel(const __grid_constant__ CUtensorMap tmX, int M, int K, int rows_per_blk,
+                           uint8_t* __restrict__ out, float* __restrict__ scale, uint8_t* __restrict__ zero,
+                           unsigned long long seed, unsigned int* err) {
   constexpr int HALF = G / 2;
+  constexpr int NH = G / 64;   // 64-element halves of a group, one TMA box each
   constexpr bool ASYM = (QMAX == 15);
   constexpr bool INT4 = (QMAX == 7) || ASYM;
-  constexpr int GS = group_stride<G>();
-  extern __shared__ __align__(16) uint8_t stage_mem[];
-  __shared__ unsigned int rowmax[2][MAXT];
-  __shared__ unsigned int rowmin[ASYM ? 2 : 1][ASYM ? MAXT : 1];   // order-preserving keys (ASYM)
+  extern __shared__ uint8_t stage_raw[];
+  // row maxima, three buffers: iteration it uses buffer it % 3 and clears
+  // buffer (it + 1) % 3, last read in iteration it - 2, which every thread
+  // has left once it passed the row barrier of iteration it - 1
+  __shared__ unsigned int rowmax[3][MAXT];
+  __shared__ unsigned int rowmin[ASYM ? 3 : 1][ASYM ? MAXT : 1];   // order-preserving keys (ASYM)
+  __shared__ __align__(8) uint64_t full[kStages];
 
   const int gpr = K / G;
   const int tid = threadIdx.x;
   const int lr = tid / gpr;
   const int grp = tid - lr * gpr;
-  const int stage_bytes = rows_per_blk * gpr * GS;
+  const int blk_groups = rows_per_blk * gpr;
+  // every box starts on a 1024-byte boundary (the 128-byte swizzle repeats
+  // every 8 lines), so line j of a box has its chunks permuted by j % 8
+  const uint32_t half_bytes = ((uint32_t)blk_groups * 128u + 1023u) & ~1023u;
+  const uint32_t stage_bytes = half_bytes * NH;
   const int nblk = (M + rows_per_blk - 1) / rows_per_blk;
-  const uint32_t stage0 = smem_u32(stage_mem);
-  constexpr int CPG = G / 8;  // 16-byte chunks per group
+  const uint32_t stage0 = (smem_u32(stage_raw) + 1023u) & ~1023u;   // swizzled boxes: 1024-byte aligned
 
+  // block it of this CTA into its stage (thread 0)
   auto issue = [&](int it) {
     const int blk = blockIdx.x + it * gridDim.x;
-    if (blk < nblk) {
-      const long row0 = (long)blk * rows_per_blk;
-      const int rows = min(rows_per_blk, (int)(M - row0));
-      const int nchunks = rows * gpr * CPG;
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(X + row0 * K);
-      const uint32_t dst = stage0 + (uint32_t)((it % kStages) * stage_bytes);
-      for (int c = tid; c < nchunks; c += blockDim.x)
-        cp_async16(dst + (uint32_t)((c / CPG) * GS + (c % CPG) * 16), src + (long)c * 16);
+    if (blk >= nblk) return;
+    const int s = it % kStages;
+    const uint32_t dst = stage0 + (uint32_t)s * stage_bytes;
+    const int g0 = blk * blk_groups;
+    mbar_arrive_expect_tx(&full[s], (uint32_t)(NH * blk_groups * 128));   // the boxes' bytes, not the padding
+    if (NH == 1) {
+      tma_load_2d(dst, &tmX, 0, g0, &full[s]);
+    } else {
+      tma_load_3d(dst, &tmX, 0, 0, g0, &full[s]);
+      tma_load_3d(dst + half_bytes, &tmX, 0, 1, g0, &full[s]);
     }
-    cp_async_commit();
   };
 
   rowmax[0][tid] = 0u;
   if (ASYM) rowmin[0][tid] = 0xFFFFFFFFu;
+  if (tid == 0) {
+    prefetch_tmap(&tmX);
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
   // launched with programmatic stream serialization: wait for the previous
   // kernel of the stream (it may produce X, or still read this output)
   grid_dependency_wait();
   grid_launch_dependents();
-#pragma unroll
-  for (int it = 0; it < kStages - 1; ++it) issue(it);
+  if (tid == 0)
+    for (int it = 0; it < kStages; ++it) issue(it);
 
   for (int it = 0;; ++it) {
     const int blk = blockIdx.x + it * gridDim.x;
     if (blk >= nblk) break;
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    issue(it + kStages - 1);
+    const int stg = it % kStages;
     if (tid < rows_per_blk) {
-      rowmax[(it + 1) & 1][tid] = 0u;
-      if (ASYM) rowmin[(it + 1) & 1][tid] = 0xFFFFFFFFu;
+      rowmax[(it + 1) % 3][tid] = 0u;
+      if (ASYM) rowmin[(it + 1) % 3][tid] = 0xFFFFFFFFu;
     }
-    unsigned int* rmax = rowmax[it & 1];
-    unsigned int* rmin = rowmin[ASYM ? (it & 1) : 0];
+    unsigned int* rmax = rowmax[it % 3];
+    unsigned int* rmin = rowmin[ASYM ? (it % 3) : 0];
 
     const long row = (long)blk * rows_per_blk + lr;
     const bool active = (lr < rows_per_blk) && (row < M);
     float2 P[HALF];  // P[i] = (y_i, y_{i+HALF})
     if (active) {
-      const uint32_t gsrc = stage0 + (uint32_t)((it % kStages) * stage_bytes + tid * GS);
+      if (!mbar_wait(&full[stg], (uint32_t)(it / kStages) & 1u)) set_device_error(err, kDevErrTimeoutFull);
 #pragma unroll
-      for (int i = 0; i < G / 8; ++i) {
-        uint4 t;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(t.x), "=r"(t.y), "=r"(t.z), "=r"(t.w)
-                     : "r"(gsrc + i * 16));
-        // elements 8i .. 8i+7 of the group
-        const uint32_t wv[4] = {t.x, t.y, t.z, t.w};
+      for (int h = 0; h < NH; ++h) {
+        const uint32_t line = stage0 + (uint32_t)stg * stage_bytes + (uint32_t)h * half_bytes + (uint32_t)tid * 128u;
+        const uint32_t sw = (uint32_t)tid & 7u;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int e = 8 * i + q;
-          const float f = (q & 1) ? bf16hi(wv[q / 2]) : bf16lo(wv[q / 2]);
-          if (e < HALF) P[e].x = f;
-          else P[e - HALF].y = f;
+        for (int c = 0; c < 8; ++c) {
+          uint4 t;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(t.x), "=r"(t.y), "=r"(t.z), "=r"(t.w)
+                       : "r"(line | ((((uint32_t)c) ^ sw) << 4)));
+          // elements 64h + 8c .. 64h + 8c + 7 of the group
+          const uint32_t wv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int e = 64 * h + 8 * c + q;
+            const float f = (q & 1) ? bf16hi(wv[q / 2]) : bf16lo(wv[q / 2]);
+            if (e < HALF) P[e].x = f;
+            else P[e - HALF].y = f;
+          }
         }
       }
       if (ROT) {
@@ -320,6 +335,12 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
       }
     }
     __syncthreads();
+    // every thread has its group in registers (its row maximum above depends
+    // on all of them): the stage takes the block after next
+    if (tid == 0) {
+      fence_proxy_async_smem();
+      issue(it + kStages);
+    }
     if (!active) continue;
 
     float s;
@@ -381,7 +402,6 @@ __global__ void __launch_bounds__(MAXT, MAXT == 128 ? 3 : 1)
       dst[YCH + c] = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
-  cp_async_wait<0>();
 }
 
 // Launch shape: rows per block R (R * K/g threads, at most MAXT) and the
@@ -396,13 +416,12 @@ template <class Occ>
 bool plan_rq_shape(int M, int K, int G, int maxt, int sms, Occ&& per_sm_of, RqShape& out) {
   const int gpr = K / G;
   const int max_r = gpr >= maxt ? 1 : maxt / gpr;
-  const int pitch = 2 * G + 16;   // group_stride<G>()
   double best = 1e30;
   bool found = false;
   for (int r = max_r; r >= 1; --r) {
     const int threads = ((r * gpr + 31) / 32) * 32;
     if (threads > maxt) continue;
-    const int smem = kStages * r * gpr * pitch;
+    const int smem = kStages * (G / 64) * ((r * gpr * 128 + 1023) / 1024) * 1024 + 1024;   // stages + alignment slack
     int per_sm = 0;
     if (!per_sm_of(threads, smem, per_sm)) return false;
     per_sm = per_sm < 1 ? 1 : per_sm;
@@ -439,13 +458,16 @@ template <int G, bool ROT, int QMAX, int MAXT, bool SR = false>
 cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* scale, uint8_t* zero,
                         unsigned long long seed, cudaStream_t st) {
   auto kern = rotate_quantize_kernel<G, ROT, QMAX, MAXT, SR>;
+  unsigned int* err = device_error_word();
+  if (!err) return cudaErrorInvalidDevicePointer;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static DeviceFlags attr_set;   // one per instantiation
   if (!attr_set.done(dev)) {
     // the largest ring any shape uses (MAXT threads' groups, kStages deep)
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStages * MAXT * group_stride<G>());
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kStages * (G / 64) * ((MAXT * 128 + 1023) / 1024) * 1024 + 1024);
     if (e != cudaSuccess) return e;
     attr_set.set(dev);
   }
@@ -459,6 +481,24 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
     }, v);
   });
   if (!ok) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+  // X as [M * K/G groups][G/64 halves][64 elements] bf16; one box per half
+  // holds the groups of one block of rows
+  CUtensorMap tm;
+  const uint64_t groups = (uint64_t)M * (uint64_t)(K / G);
+  const uint32_t blk_groups = (uint32_t)(sh.rows_per_blk * (K / G));
+  bool enc;
+  if (G == 64) {
+    const uint64_t dims[2] = {64, groups};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, blk_groups};
+    enc = make_tmap_nd(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    const uint64_t dims[3] = {64, 2, groups};
+    const uint64_t strides[2] = {128, 256};
+    const uint32_t box[3] = {64, 1, blk_groups};
+    enc = make_tmap_nd(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (!enc) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sh.grid, 1, 1);
   cfg.blockDim = dim3(sh.threads, 1, 1);
@@ -469,7 +509,7 @@ cudaError_t launch_rq_t(const uint16_t* X, int M, int K, uint8_t* out, float* sc
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, X, M, K, sh.rows_per_blk, out, scale, zero, seed);
+  e = cudaLaunchKernelEx(&cfg, kern, tm, M, K, sh.rows_per_blk, out, scale, zero, seed, err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
