@@ -640,18 +640,20 @@ def main():
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
-    def k1(s):
+    def k1(s, st=None):
+        st = stream if st is None else st
         if w4a8:
-            w4.w8a8_rotate_quantize_act(s["X"], g, Xq=s["Xq"], x_scale=s["xs"], stream=stream)
+            w4.w8a8_rotate_quantize_act(s["X"], g, Xq=s["Xq"], x_scale=s["xs"], stream=st)
         else:
-            w4.w4a4_rotate_quantize_act(s["X"], g, s["L1"], Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=stream)
+            w4.w4a4_rotate_quantize_act(s["X"], g, s["L1"], Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=st)
 
-    def k2(s):
+    def k2(s, st=None):
+        st = stream if st is None else st
         if w4a8:
-            w4.w4a8_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], s["wz"], g, s["bias"], Y=s["Y"], stream=stream)
+            w4.w4a8_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], s["wz"], g, s["bias"], Y=s["Y"], stream=st)
         else:
             w4.w4a4_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], g, s["T"], s["L2"], s["bias"], Y=s["Y"],
-                         stream=stream)
+                         stream=st)
 
     def step(s):
         k1(s)
@@ -710,16 +712,26 @@ def main():
     total_ms = e_start.elapsed_time(e_end)
 
     # per-kernel durations for the roofline: each kernel alone, back to back,
-    # on the same rotating sets (CUDA events on the launching stream)
+    # on the same rotating sets, replayed from a CUDA graph so that the host's
+    # per-call cost (Python and argument checks, ~10 us) does not set the
+    # pace of the short kernels (CUDA events on the replaying stream)
     def timed(fn, n):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         for i in range(3):
             fn(sets[i % len(sets)])
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(n):
+                fn(sets[i % len(sets)], torch.cuda.current_stream())
+        graph.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for i in range(n):
-            fn(sets[i % len(sets)])
+        with torch.cuda.stream(stream):
+            graph.replay()
         b.record(stream)
         torch.cuda.synchronize()
+        del graph
         return a.elapsed_time(b) / n
 
     n_split = min(args.steps, 200)
@@ -817,7 +829,8 @@ def main():
                        "bias": spec.bias, "parallelism": f"replicas x{world} (token shards, no exchange)",
                        "l2": f"{args.sets} rotating input sets (> L2)",
                        "clock_soak_ms": args.soak_ms},
-            "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3, "note": "each kernel timed alone, back to back"},
+            "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3,
+                         "note": "each kernel timed alone, back to back, replayed from a CUDA graph"},
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
                          "frac": k2_tops / int8_peak,
                          "frac_clock_adjusted": (k2_tops / adj) if adj else None,

@@ -134,6 +134,7 @@ struct Cfg {
   static_assert(PS % kSets == 0, "each widen set owns its packed stages");
   static_assert(US >= kSets && kLead >= 1, "widened ring");
   static_assert(kWOff % 1024 == 0 && kAOff % 1024 == 0, "128-byte swizzle atoms");
+  static_assert(kWOff + US * kWideB <= kRing && (MODE != 2 || kAOff + AS * kI8A <= kRing), "rings inside the ring area");
   static_assert(!LR || MODE == 1, "low-rank branch: W4A4 only");
   static_assert(!LR || kOutStageBytes <= kLrBytes, "epilogue staging inside the low-rank buffer");
 };
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (lane == 0) {
             if (MODE == 1) {
-              const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
+              const uint32_t b_stage = sbase + (uint32_t)(C::kWOff + s * C::kWideB);
 #pragma unroll
               for (int ks = 0; ks < BK / 32; ++ks)
                 mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8),
@@ -457,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_commit_pair_mc(&bar->empty[s], 0x3);
             } else if (MODE == 2) {
               const uint32_t a_stage = sbase + (uint32_t)(C::kAOff + ps * C::kI8A);
-              const uint32_t b_stage = sbase + (uint32_t)(PS * C::kPkStage + s * C::kWideB);
+              const uint32_t b_stage = sbase + (uint32_t)(C::kWOff + s * C::kWideB);
 #pragma unroll
               for (int ks = 0; ks < BK / 32; ++ks)
                 mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
@@ -621,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (has_b) {
         const uint32_t row =
-            sbase + (uint32_t)(PS * C::kPkStage + u * C::kWideB + (r >> 3) * 1024 + (r & 7) * 128);
+            sbase + (uint32_t)(C::kWOff + u * C::kWideB + (r >> 3) * 1024 + (r & 7) * 128);
         const uint32_t rsw128 = (uint32_t)(r & 7);
         uint32_t zk = 0;
         if constexpr (MODE == 2) {
