@@ -52,9 +52,8 @@ def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
 # they were taken from (sha256 prefix); reported as null once the source
 # changes.
 MEASURED_TRAFFIC = {
-    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6488a2c765a2d4a6", 11.880448e6 + 0.030464e6),
-    "gemm_w4a8": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6488a2c765a2d4a6", 18.960384e6 + 0.091648e6),
-    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "61d3e84e299a0ca7", 28.377344e6),
+    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "d0282a6d1240b6c0", 11.910e6),
+    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "59bbaf52c3e58355", 28.378e6),
 }
 
 
@@ -252,9 +251,8 @@ def run_mlp(args):
                          hs=torch.empty((M,), dtype=torch.float32, device="cuda"),
                          Th=torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
                          Y=torch.empty((M, D), dtype=torch.bfloat16, device="cuda")))
-    stream = torch.cuda.current_stream()
-
     def step(s, fused=True):
+        stream = torch.cuda.current_stream()
         w4.w4a4_rotate_quantize_act(s["X"], g, L1u, Xq=s["Xq"], x_scale=s["xs"], T=s["T"], stream=stream)
         if fused:
             w4.w4a4_gemm_gelu(s["Xq"], s["xs"], Wq_u, ws_u, g, s["T"], L2u, bu, Y=s["h"], stream=stream)
@@ -265,15 +263,22 @@ def run_mlp(args):
         w4.w4a4_gemm(s["hq"], s["hs"], Wq_d, ws_d, g, s["Th"], L2d, bd, Y=s["Y"], stream=stream)
 
     def timed(fused, n):
+        # n steps captured in a CUDA graph and replayed
         for i in range(args.warmup):
             step(sets[i % 2], fused)
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(n):
-            step(sets[i % 2], fused)
-        e1.record(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(n):
+                step(sets[i % 2], fused)
+        graph.replay()
         torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del graph
         return e0.elapsed_time(e1) / n
 
     clocks = ClockSampler(0)
@@ -395,15 +400,23 @@ def run_block(args):
                            workspace=L["wsp"])
 
     def timed(fn, n):
+        # n calls captured in a CUDA graph and replayed (host time per call
+        # would otherwise pace the small layers)
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(n):
+                fn()
+        graph.replay()
+        torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for _ in range(n):
-            fn()
+        graph.replay()
         e1.record()
         torch.cuda.synchronize()
+        del graph
         return e0.elapsed_time(e1) / n * 1e3
 
     per = {L["spec"].name: timed(lambda L=L: run(L), args.steps) for L in layers}
@@ -467,19 +480,39 @@ def run_sweep(args):
         X[:, ch[: max(1, round(0.01 * K))]] *= 100.0
         return X.to(torch.bfloat16)
 
+    def graph_of(fn, with_flush):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if with_flush:
+                flush.fill_(1)
+            if fn is not None:
+                fn(torch.cuda.current_stream())
+        return g
+
+    def replay_us(g, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g.replay()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / n
+
+    g_flush = graph_of(None, True)
+
     def timed(fn):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        # the layer call and a 256 MB L2 flush replayed from one CUDA graph,
+        # back to back (no host time between calls), minus the flush alone
         for _ in range(args.warmup):
-            fn()
-        ts = []
-        for _ in range(args.steps):
-            flush.fill_(1)
-            ev[0].record(stream)
-            fn()
-            ev[1].record(stream)
-            ev[1].synchronize()
-            ts.append(ev[0].elapsed_time(ev[1]) * 1e3)
-        return statistics.median(ts)
+            fn(stream)
+        torch.cuda.synchronize()
+        g = graph_of(fn, True)
+        n = max(args.steps, 5)
+        us = min(replay_us(g, n) - replay_us(g_flush, n) for _ in range(3))
+        del g
+        return us
 
     def emit(name, M, K, N, g, r, variant, us, code_bytes):
         ops = 2.0 * M * N * K
@@ -492,7 +525,7 @@ def run_sweep(args):
                           "frac_of_int8_nominal": ops / (us * 1e-6) / 1e12 / INT8_NOMINAL_TOPS,
                           "frac_of_int8_measured": ops / (us * 1e-6) / 1e12 / i8,
                           "roofline_us": roof_us, "frac_of_roofline": roof_us / us,
-                          "l2": "flushed before every call"}), flush=True)
+                          "l2": "flushed before every call (the flush time is subtracted)"}), flush=True)
 
     # the tiny single layer
     X = acts(64, 256, 0)
@@ -500,7 +533,7 @@ def run_sweep(args):
     L1, L2 = draw((256, 16), 2, 0.01), draw((16, 256), 3, 0.01)
     ws_buf = torch.empty((w4.w4a4_workspace_bytes(64, 256, 16),), dtype=torch.uint8, device="cuda")
     Y = torch.empty((64, 256), dtype=torch.bfloat16, device="cuda")
-    us = timed(lambda: w4.w4a4_linear(X, Wq, ws, 64, L1, L2, None, Y=Y, workspace=ws_buf))
+    us = timed(lambda st: w4.w4a4_linear(X, Wq, ws, 64, L1, L2, None, Y=Y, workspace=ws_buf, stream=st))
     emit("tiny", 64, 256, 256, 64, 16, "w4a4", us, 64 * 128)
 
     Ms = [256, 1024, 4608, 9216, 16384]
@@ -521,11 +554,11 @@ def run_sweep(args):
                 L1 = L1f[:, :r].contiguous() if r else None
                 L2 = L2f[:r].contiguous() if r else None
                 wsb = torch.empty((w4.w4a4_workspace_bytes(M, K, r),), dtype=torch.uint8, device="cuda")
-                us = timed(lambda: w4.w4a4_linear(X, Wq, ws, 128, L1, L2, b, Y=Y, workspace=wsb))
+                us = timed(lambda st: w4.w4a4_linear(X, Wq, ws, 128, L1, L2, b, Y=Y, workspace=wsb, stream=st))
                 emit("c5", M, K, N, 128, r, "w4a4", us, M * K // 2)
                 del wsb
             wsb = torch.empty((w4.w4a8_workspace_bytes(M, K),), dtype=torch.uint8, device="cuda")
-            us = timed(lambda: w4.w4a8_linear(X, Wq8, ws8, wz8, 128, b, Y=Y, workspace=wsb))
+            us = timed(lambda st: w4.w4a8_linear(X, Wq8, ws8, wz8, 128, b, Y=Y, workspace=wsb, stream=st))
             emit("c5", M, K, N, 128, 0, "w4a8", us, M * K)
             del X, Y, wsb
             torch.cuda.empty_cache()
@@ -834,7 +867,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
                          "frac": k2_tops / int8_peak,
                          "frac_clock_adjusted": (k2_tops / adj) if adj else None,
-                         "traffic": _traffic("gemm_w4a8" if w4a8 else "gemm", spec.name),
+                         "traffic": None if w4a8 else _traffic("gemm", spec.name),
                          "peak_note": f"int8 = 2 x {pk['source']} burst bf16 {pk['bf16']} TFLOP/s (kernel timed "
                                       f"alone); {2.0 * pk['bf16_sustained']:.0f} with the sustained figure"},
             "roofline_k1": {"bound": "hbm", "achieved": k1_bytes / (k1 * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
