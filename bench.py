@@ -669,6 +669,8 @@ def main():
                  xs=torch.empty((M,), dtype=torch.float32, device="cuda"),
                  T=torch.empty((M, r), dtype=torch.bfloat16, device="cuda") if r else None,
                  Y=torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
+        s["work"] = torch.empty((w4.w4a8_workspace_bytes(M, K) if w4a8 else w4.w4a4_workspace_bytes(M, K, r),),
+                                dtype=torch.uint8, device="cuda")
         sets.append(s)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -689,8 +691,14 @@ def main():
                          stream=st)
 
     def step(s):
-        k1(s)
-        k2(s)
+        # one whole layer through the public call (its kernels: rotate +
+        # quantize, the low-rank down-projection when r > 0, the GEMM)
+        if w4a8:
+            w4.w4a8_linear(s["X"], s["Wq"], s["ws"], s["wz"], g, s["bias"], Y=s["Y"], workspace=s["work"],
+                           stream=stream)
+        else:
+            w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"], workspace=s["work"],
+                           stream=stream)
 
     for i in range(args.warmup):
         step(sets[i % len(sets)])
@@ -867,12 +875,12 @@ def main():
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
                          "frac": k2_tops / int8_peak,
                          "frac_clock_adjusted": (k2_tops / adj) if adj else None,
-                         "traffic": None if w4a8 else _traffic("gemm", spec.name),
+                         "traffic": None if (w4a8 or r) else _traffic("gemm", spec.name),
                          "peak_note": f"int8 = 2 x {pk['source']} burst bf16 {pk['bf16']} TFLOP/s (kernel timed "
                                       f"alone); {2.0 * pk['bf16_sustained']:.0f} with the sustained figure"},
             "roofline_k1": {"bound": "hbm", "achieved": k1_bytes / (k1 * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": k1_bytes / (k1 * 1e-3) / 1e9 / pk["hbm_gbs"],
-                            "traffic": None if w4a8 else _traffic("rotate_quantize", spec.name)},
+                            "traffic": None if (w4a8 or r) else _traffic("rotate_quantize", spec.name)},
             "gpu_launches": 2 * args.steps + (args.steps if r else 0),
             "clocks": clk, "wall_s": wall, "e2e": e2e,
         }
