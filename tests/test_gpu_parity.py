@@ -117,6 +117,8 @@ GEMM_CASES = [
     (96, 512, 12288, 128, 128, False),  # long K
     (300, 640, 1024, 64, 144, False),   # two low-rank chunks, the second 16 ranks
     (2048, 3072, 256, 128, 256, True),  # rank 256 and more tiles than pairs: buffer hand-off across tiles
+    (512, 3072, 3072, 128, 0, True),    # few tiles: split-K over two pairs per tile
+    (256, 1024, 12288, 64, 0, False),   # split-K over four pairs per tile, long K
 ]
 
 
@@ -285,6 +287,25 @@ def test_w4a4_layer_with_fused_gelu(M, N, K, g, r):
     Y2 = w4.w4a4_linear_gelu(X, Wq, ws, g, L1, L2, b)
     torch.cuda.synchronize()
     assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+
+
+@pytest.mark.parametrize("K,act", [(3072, False), (3072, True), (12288, False)])
+def test_split_k_equals_the_persistent_form(K, act):
+    """A layer with few tiles runs in the split-K form (its K range spread
+    over a cluster of pairs, int32 partials summed through distributed shared
+    memory).  Quantization is per token, so the first 256 rows of a large
+    layer (many tiles: the persistent form) must come out bit for bit the
+    same as those rows run on their own."""
+    import torch
+    M, N, g = 4608, 3072, 128
+    d = _layer(M, N, K, g, 0, True, seed=K + (7 if act else 3))
+    X, W, b = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    Wq, ws = w4.w4a4_quantize_weights(W, g)
+    lin = w4.w4a4_linear_gelu if act else w4.w4a4_linear
+    Y_all = lin(X, Wq, ws, g, None, None, b)
+    Y_few = lin(X[:256].contiguous(), Wq, ws, g, None, None, b)
+    torch.cuda.synchronize()
+    assert torch.equal(Y_few.view(torch.int16), Y_all[:256].view(torch.int16))
 
 
 def test_fused_mlp_chain():

@@ -86,6 +86,7 @@ constexpr uint32_t kACol0 = 256; // A ring: 32 columns per stage
 constexpr int kStageTile = 32 * 32 * 2;            // epilogue staging tile: 32 x 32 bf16
 constexpr int kOutStageBytes = 16 * kStageTile;    // one per epilogue warp
 constexpr int kBarBytes = 512;
+constexpr int kPartPitch = 256 * 4 + 16;           // split-K: int32 partial row pitch (bank-spread)
 
 // MODE 0: W8A8 (int8 x int8, TMA straight into the MMA layout); 1: W4A4
 // (packed INT4 x packed INT4, both widened, A into TMEM); 2: W4A8 (the int8
@@ -142,6 +143,7 @@ struct Cfg {
 struct Params {
   GemmArgs a;
   unsigned int* err;
+  int split;   // split-K form: K slices (pairs per cluster), else 1
 };
 
 struct Barriers {
@@ -231,7 +233,13 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return 0.5f * x * (1.0f + tanhf(u));
 }
 
-template <int MODE, bool LR, bool ACT>
+// SPLIT (W4A4 without the low-rank branch): a cluster of prm.split pairs
+// shares one 256 x 256 tile; pair q accumulates the k-blocks
+// [q nk / split, (q + 1) nk / split), every CTA leaves its int32 partial in
+// shared memory, and after a cluster barrier CTA (q, half) sums column slice
+// q of its half over all pairs (exact integer sums, in pair order) and runs
+// the epilogue on it.  For layers with too few tiles to occupy the GPU.
+template <int MODE, bool LR, bool ACT, bool SPLIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
@@ -249,16 +257,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   Barriers* bar = reinterpret_cast<Barriers*>(smem_raw + (sbase - raw) + C::kDataBytes);
 
+  static_assert(!SPLIT || (MODE == 1 && !LR), "split-K form: W4A4 without the low-rank branch");
+  static_assert(!SPLIT || BM * kPartPitch <= C::kRing, "split-K partial inside the ring area");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t rank = SPLIT ? (crank & 1u) : crank;      // CTA within its pair
+  const uint32_t pbase = SPLIT ? (crank & ~1u) : 0u;       // the pair's even CTA in the cluster
+  const uint16_t pmask = (uint16_t)(0x3u << pbase);        // both CTAs of the pair
   const bool leader = rank == 0;
   const int n_tiles = (p.N + BN - 1) / BN;
   const int total_tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * n_tiles;
-  const int pair0 = blockIdx.x >> 1;
-  const int pair_stride = gridDim.x >> 1;
+  const int pair0 = SPLIT ? (int)(blockIdx.x / (2 * prm.split)) : (int)(blockIdx.x >> 1);
+  const int pair_stride = SPLIT ? total_tiles : (int)(gridDim.x >> 1);
   const int my_tiles = pair0 < total_tiles ? (total_tiles - pair0 + pair_stride - 1) / pair_stride : 0;
-  const int nk = p.K / BK;
+  // k-blocks of this pair: all of them, or its slice in the split-K form
+  const int kb0 = SPLIT ? (int)(crank >> 1) * (p.K / BK) / prm.split : 0;
+  const int nk = SPLIT ? ((int)(crank >> 1) + 1) * (p.K / BK) / prm.split - kb0 : p.K / BK;
   const int lr_chunks = LR ? (p.rank + LRC - 1) / LRC : 0;
   // tile i of this pair (i < my_tiles): this CTA's rows, the pair's columns
   auto tile_m = [&](int i) { return ((pair0 + i * pair_stride) / n_tiles) * (2 * BM) + (int)rank * BM; };
@@ -374,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = sbase + (uint32_t)(s * kStageBytes);
           mbar_arrive_expect_tx(&bar->tma_full[s], (uint32_t)kStageBytes);
-          if (MODE != 2) tma_load_2d(dst, &tmA, kb * kColA, row_a, &bar->tma_full[s]);
-          tma_load_2d(dst + kABytes, &tmB, kb * kColB, row_b, &bar->tma_full[s]);
+          if (MODE != 2) tma_load_2d(dst, &tmA, (kb0 + kb) * kColA, row_a, &bar->tma_full[s]);
+          tma_load_2d(dst + kABytes, &tmB, (kb0 + kb) * kColB, row_b, &bar->tma_full[s]);
           if (++s == NS) { s = 0; ph ^= 1u; }
           if constexpr (MODE == 2) {
             // the int8 A tile into its own ring, once the MMAs have freed the slot
@@ -385,7 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&bar->a_full[as], (uint32_t)C::kI8A);
-            tma_load_2d(sbase + (uint32_t)(C::kAOff + as * C::kI8A), &tmA, kb * BK, row_a, &bar->a_full[as]);
+            tma_load_2d(sbase + (uint32_t)(C::kAOff + as * C::kI8A), &tmA, (kb0 + kb) * BK, row_a,
+                        &bar->a_full[as]);
             if (++as == C::AS) { as = 0; a_ph ^= 1u; }
           }
           if (LR && kb == nk / 2) lr_eligible = (i + 1) * lr_chunks;
@@ -414,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_remote(&bar->full[s], 0);
+            mbar_arrive_remote(&bar->full[s], pbase);
             if (++s == S8) { s = 0; ph ^= 1u; }
           }
         }
@@ -424,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_remote(&bar->lr_ready, 0);
+          mbar_arrive_remote(&bar->lr_ready, pbase);
         }
       }
     }
@@ -455,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_i8_ts_pair(tmem + kAccCol, tmem + kACol0 + (uint32_t)(s * (BK / 4) + ks * 8),
                                smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
                                (kb | ks) != 0 ? 1u : 0u);
-              tc_commit_pair_mc(&bar->empty[s], 0x3);
+              tc_commit_pair_mc(&bar->empty[s], pmask);
             } else if (MODE == 2) {
               const uint32_t a_stage = sbase + (uint32_t)(C::kAOff + ps * C::kI8A);
               const uint32_t b_stage = sbase + (uint32_t)(C::kWOff + s * C::kWideB);
@@ -464,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
                                smem_desc_kmajor_sw128(b_stage + (uint32_t)(ks * 32)), idesc,
                                (kb | ks) != 0 ? 1u : 0u);
-              tc_commit_pair_mc(&bar->empty[s], 0x3);
-              tc_commit_pair_mc(&bar->a_empty[ps], 0x3);
+              tc_commit_pair_mc(&bar->empty[s], pmask);
+              tc_commit_pair_mc(&bar->a_empty[ps], pmask);
             } else {
               const uint32_t a_stage = sbase + (uint32_t)(s * C::kI8Stage);
 #pragma unroll
@@ -473,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_i8_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_stage + (uint32_t)(ks * 32)),
                                smem_desc_kmajor_sw128(a_stage + C::kI8A + (uint32_t)(ks * 32)), idesc,
                                (kb | ks) != 0 ? 1u : 0u);
-              tc_commit_pair_mc(&bar->tma_empty[s], 0x3);
+              tc_commit_pair_mc(&bar->tma_empty[s], pmask);
             }
           }
           __syncwarp();
@@ -481,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++ps == (MODE == 2 ? C::AS : PS)) ps = 0;
         }
         // the integer product of the tile is complete
-        if (ok && lane == 0) tc_commit_pair_mc(&bar->acc_full, 0x3);
+        if (ok && lane == 0) tc_commit_pair_mc(&bar->acc_full, pmask);
         __syncwarp();
         if (LR) {
           // Once both epilogues have rewritten the accumulator as fp32
@@ -504,17 +520,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_bf16_ss_pair(tmem + kAccCol, smem_desc_kmajor_sw128(a_addr),
                                  smem_desc_mnmajor_sw128(b_addr, (uint32_t)(C::kLrL2 / 2), 1024), idesc_lr, 1u);
               }
-              if (c + 1 < lr_chunks) tc_commit_pair_mc(&bar->lr_empty, 0x3);
+              if (c + 1 < lr_chunks) tc_commit_pair_mc(&bar->lr_empty, pmask);
             }
             __syncwarp();
           }
-          if (ok && lane == 0) tc_commit_pair_mc(&bar->lr_done, 0x3);
+          if (ok && lane == 0) tc_commit_pair_mc(&bar->lr_done, pmask);
         }
         __syncwarp();
       }
       // drain: every MMA issued so far has completed before teardown
       if (lane == 0) {
-        tc_commit_pair_mc(&bar->drain, 0x1);
+        tc_commit_pair_mc(&bar->drain, (uint16_t)(0x1u << pbase));
         if (!mbar_wait(&bar->drain, 0)) set_device_error(prm.err, kDevErrTimeoutDrain);
       }
       __syncwarp();
@@ -656,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(&bar->full[u], 0);
+      if (lane == 0) mbar_arrive_remote(&bar->full[u], pbase);
       return true;
     };
 
@@ -727,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(&bar->conv, 0);
+        if (lane == 0) mbar_arrive_remote(&bar->conv, pbase);
         if (!mbar_wait(&bar->lr_done, (uint32_t)i & 1u)) set_device_error(prm.err, kDevErrTimeoutAcc);
         tc_fence_after();
       }
@@ -736,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(&bar->acc_empty, 0);
+      if (lane == 0) mbar_arrive_remote(&bar->acc_empty, pbase);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const int c0 = cq * C::kColsPerWarp + ch * 32;
@@ -790,7 +806,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 
-    if (!PACKED) {
+    if constexpr (SPLIT) {
+      // one tile: widen this pair's k-blocks, then leave this warp's share
+      // of the int32 partial (32 rows x 64 columns) in the ring area, idle
+      // once the accumulator is final (every MMA has read its stages)
+      for (int g = set; g < total_kb; g += kSets)
+        if (!widen(g)) break;
+      if (my_tiles > 0) {
+        if (!mbar_wait(&bar->acc_full, 0u)) set_device_error(prm.err, kDevErrTimeoutAcc);
+        tc_fence_after();
+        uint32_t v[2][32];
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(cq * C::kColsPerWarp) + kAccCol;
+        tmem_ld_32x32b_x32(taddr, v[0]);
+        tmem_ld_32x32b_x32(taddr + 32, v[1]);
+        tmem_wait_ld();
+        const uint32_t prow = sbase + (uint32_t)(r * kPartPitch + cq * C::kColsPerWarp * 4);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            st_shared_v4(prow + (uint32_t)((ch * 32 + 4 * q) * 4),
+                         make_uint4(v[ch][4 * q], v[ch][4 * q + 1], v[ch][4 * q + 2], v[ch][4 * q + 3]));
+      }
+    } else if (!PACKED) {
       for (int i = 0; i < my_tiles; ++i) epilogue(i);
     } else {
       // The epilogue of tile i-1 runs before this warp widens any k-block
@@ -816,6 +854,74 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncwarp();   // single-lane roles rejoin their warps before the aligned cluster barrier
   cluster_sync();
+  if constexpr (SPLIT) {
+    if (warp < 16 && my_tiles > 0) {
+      // column slice q of this CTA's 128 rows: the pairs' partials summed in
+      // pair order (exact int32), then the epilogue of the unsplit form.  A
+      // thread keeps one group of four columns (their scales and bias in
+      // registers) and walks rows `step` apart, two rows' loads in flight.
+      const int S = prm.split;
+      const int per_row = BN / S / 4;                    // column groups in the slice
+      const int step = 16 * 32 / per_row;                // rows per pass
+      const int c = (int)(crank >> 1) * (BN / S) + (threadIdx.x % per_row) * 4;
+      const int n = tile_n(0) + c;
+      const int row0 = threadIdx.x / per_row;
+      if (n < p.N) {
+        float sw[4], bv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sw[j] = __ldg(p.b_scale + n + j) * p.inv_group;
+          bv[j] = p.bias ? bf16_bits_to_float(__ldg(p.bias + n + j)) : 0.0f;
+        }
+        for (int rb = row0; rb < BM; rb += 2 * step) {
+          uint4 w[2][4];
+          float sa[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int row = rb + k * step;
+            const long m = (long)tile_m(0) + row;
+            sa[k] = (row < BM && m < p.M) ? __ldg(p.a_scale + m) : 0.0f;
+            const uint32_t local = sbase + (uint32_t)(row * kPartPitch + c * 4);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q < S && row < BM) w[k][q] = ld_cluster_v4(map_to_rank(local, (uint32_t)(2 * q) + rank));
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int row = rb + k * step;
+            const long m = (long)tile_m(0) + row;
+            if (row >= BM || m >= p.M) continue;
+            uint32_t acc[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (q < S) {
+                acc[0] += w[k][q].x;
+                acc[1] += w[k][q].y;
+                acc[2] += w[k][q].z;
+                acc[3] += w[k][q].w;
+              }
+            }
+            if (p.acc_debug)
+              *reinterpret_cast<uint4*>(p.acc_debug + m * p.N + n) =
+                  make_uint4((uint32_t)((int)acc[0] >> kShift), (uint32_t)((int)acc[1] >> kShift),
+                             (uint32_t)((int)acc[2] >> kShift), (uint32_t)((int)acc[3] >> kShift));
+            float y[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              y[j] = __fadd_rn(__fmul_rn(__fmul_rn(acc_to_float<true>(acc[j]), sa[k]), sw[j]), bv[j]);
+              if constexpr (ACT) y[j] = gelu_tanh(y[j]);
+            }
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
+            *reinterpret_cast<uint2*>(p.Y + m * p.N + n) =
+                make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync();   // the partials stay readable until every CTA has summed its slice
+  }
   if (warp == kTmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols);
@@ -823,10 +929,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
-template <int MODE, bool LR, bool ACT = false>
-cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
+// split > 1 (SPLIT): one cluster of `split` pairs per tile, all resident at once.
+template <int MODE, bool LR, bool ACT = false, bool SPLIT = false>
+cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st, int split = 1) {
   using C = Cfg<MODE, LR>;
-  auto kern = gemm_kernel<MODE, LR, ACT>;
+  auto kern = gemm_kernel<MODE, LR, ACT, SPLIT>;
   static DeviceFlags configured;   // one per instantiation
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -863,20 +970,21 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
   int sms = 0;
   if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * std::min(pairs, sms / 2), 1, 1);   // persistent: one pair per TPC
+  // persistent: one pair per TPC; split-K: one cluster of `split` pairs per tile
+  cfg.gridDim = dim3(SPLIT ? 2 * split * pairs : 2 * std::min(pairs, sms / 2), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.x = SPLIT ? 2 * split : 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  Params prm{a, err};
+  Params prm{a, err, SPLIT ? split : 1};
   e = cudaLaunchKernelEx(&cfg, kern, prm, tA, tB, tY, tT, tL2);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -886,11 +994,74 @@ cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st) {
 
 unsigned int* device_error_word();
 
+namespace {
+
+// K slices for the split-K form of a W4A4 layer without the low-rank branch:
+// 4 or 2 when the layer has too few 256 x 256 tiles to give every TPC one
+// (tiles x slices <= SMs / 2), each slice keeps at least two k-blocks, and
+// every cluster of 2 x slices CTAs fits on the GPU at once; else 1 (the
+// persistent form).
+struct SplitKey {
+  int64_t v[4];
+};
+template <bool ACT>
+cudaError_t plan_split(const GemmArgs& a, int* split) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int sms = 0;
+  if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
+  const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + 255) / 256);
+  const int nkb = a.K / BK;
+  static PlanCache<SplitKey, int, 32> cache;
+  const SplitKey key = {{dev, tiles, nkb, sms}};
+  const bool ok = cache.get(key, *split, [&](int& out) {
+    out = 1;
+    using C = Cfg<1, false>;
+    auto kern = gemm_kernel<1, false, ACT, true>;
+    for (int s : {4, 2}) {
+      if (tiles * s > sms / 2 || nkb < 2 * s) continue;
+      if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes)) !=
+          cudaSuccess)
+        return false;
+      cudaLaunchConfig_t qc = {};
+      qc.gridDim = dim3(2 * s * tiles, 1, 1);
+      qc.blockDim = dim3(kThreads, 1, 1);
+      qc.dynamicSmemBytes = C::kSmemBytes;
+      cudaLaunchAttribute qa;
+      qa.id = cudaLaunchAttributeClusterDimension;
+      qa.val.clusterDim.x = 2 * s;
+      qa.val.clusterDim.y = 1;
+      qa.val.clusterDim.z = 1;
+      qc.attrs = &qa;
+      qc.numAttrs = 1;
+      int clusters = 0;
+      if ((e = cudaOccupancyMaxActiveClusters(&clusters, kern, &qc)) != cudaSuccess) return false;
+      if (clusters >= tiles) {
+        out = s;
+        break;
+      }
+    }
+    return true;
+  });
+  return ok ? cudaSuccess : e;
+}
+
+}  // namespace
+
 cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st) {
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorInvalidDevicePointer;
   if (mode == GemmMode::kW8A8) return launch_impl<0, false>(a, err, st);
   if (mode == GemmMode::kW4A8) return launch_impl<2, false>(a, err, st);
+  if (a.rank == 0) {
+    int split = 1;
+    cudaError_t e = a.act == 1 ? plan_split<true>(a, &split) : plan_split<false>(a, &split);
+    if (e != cudaSuccess) return e;
+    if (split > 1)
+      return a.act == 1 ? launch_impl<1, false, true, true>(a, err, st, split)
+                        : launch_impl<1, false, false, true>(a, err, st, split);
+  }
   if (a.act == 1)
     return a.rank > 0 ? launch_impl<1, true, true>(a, err, st) : launch_impl<1, false, true>(a, err, st);
   return a.rank > 0 ? launch_impl<1, true>(a, err, st) : launch_impl<1, false>(a, err, st);

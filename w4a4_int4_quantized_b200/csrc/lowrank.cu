@@ -48,23 +48,6 @@ struct LrParams {
   int withhold;                 // self-test: the producer issues no operand load
 };
 
-// A 16-byte load from a cluster peer's shared memory, without a compiler
-// memory barrier, so that independent loads can be in flight together (the
-// partials are not written again before the kernel's closing cluster barrier).
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     lowrank_down_kernel(const LrParams p, const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmL1) {
