@@ -52,16 +52,17 @@ def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
 # they were taken from (sha256 prefix); reported as null once the source
 # changes.
 MEASURED_TRAFFIC = {
-    "gemm": ("w4a4_int4_quantized_b200/csrc/gemm.cu", "d0282a6d1240b6c0", 11.910e6),
-    "rotate_quantize": ("w4a4_int4_quantized_b200/csrc/quantize.cu", "59bbaf52c3e58355", 28.378e6),
+    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "aa2f8d50d44e83ee", 11.899e6),
+    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "aa2f8d50d44e83ee", 20.498e6),
+    ("rotate_quantize", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/quantize.cu", "59bbaf52c3e58355", 28.378e6),
 }
 
 
 def _traffic(kernel: str, workload: str):
-    if workload != "attn_proj":
+    if (kernel, workload) not in MEASURED_TRAFFIC:
         return None
     import hashlib
-    path, sha, value = MEASURED_TRAFFIC[kernel]
+    path, sha, value = MEASURED_TRAFFIC[(kernel, workload)]
     try:
         with open(os.path.join(ROOT, path), "rb") as f:
             cur = hashlib.sha256(f.read()).hexdigest()[:16]

@@ -76,6 +76,10 @@ WORKLOADS: dict[str, LayerSpec] = {
     "block_first_w8a8": LayerSpec("block_first_w8a8", 9216, 3072, 3072, 128, w8a8=True, seed=4),
     "block_last_w8a8": LayerSpec("block_last_w8a8", 9216, 3072, 3072, 128, w8a8=True, seed=4),
     "block_tmlp_w8a8": LayerSpec("block_tmlp_w8a8", 2, 256, 3072, 128, w8a8=True, seed=4),
+    # a point of the shape sweep: the MLP down-projection shape at 256 tokens,
+    # too few tiles for the persistent GEMM (it runs in the split-K form)
+    "m256_down": LayerSpec("m256_down", 256, 12288, 3072, 128, rank=0, bias=True, seed=1043,
+                           outlier_scale=100.0),
 }
 
 
