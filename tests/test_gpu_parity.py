@@ -119,6 +119,9 @@ GEMM_CASES = [
     (2048, 3072, 256, 128, 256, True),  # rank 256 and more tiles than pairs: buffer hand-off across tiles
     (512, 3072, 3072, 128, 0, True),    # few tiles: split-K over two pairs per tile
     (256, 1024, 12288, 64, 0, False),   # split-K over four pairs per tile, long K
+    (1, 3072, 3072, 128, 0, True),      # split-K with a single token row
+    (40, 8, 3072, 128, 0, False),       # split-K, one tile holding 8 of its 256 columns
+    (256, 1024, 12288, 128, 32, True),  # split-K with the low-rank term in the reduction
 ]
 
 

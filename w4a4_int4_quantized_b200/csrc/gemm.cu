@@ -87,6 +87,7 @@ constexpr int kStageTile = 32 * 32 * 2;            // epilogue staging tile: 32 
 constexpr int kOutStageBytes = 16 * kStageTile;    // one per epilogue warp
 constexpr int kBarBytes = 512;
 constexpr int kPartPitch = 256 * 4 + 16;           // split-K: int32 partial row pitch (bank-spread)
+constexpr int kTOff = 128 * kPartPitch;            // split-K: T rows after the partials (ring area)
 
 // MODE 0: W8A8 (int8 x int8, TMA straight into the MMA layout); 1: W4A4
 // (packed INT4 x packed INT4, both widened, A into TMEM); 2: W4A8 (the int8
@@ -233,13 +234,14 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return 0.5f * x * (1.0f + tanhf(u));
 }
 
-// SPLIT (W4A4 without the low-rank branch): a cluster of prm.split pairs
-// shares one 256 x 256 tile; pair q accumulates the k-blocks
+// SPLIT 1 (W4A4) or 2 (W4A4 with a small low-rank branch, its term added in
+// the reduction): a cluster of prm.split pairs shares one 256 x 256 tile;
+// pair q accumulates the k-blocks
 // [q nk / split, (q + 1) nk / split), every CTA leaves its int32 partial in
 // shared memory, and after a cluster barrier CTA (q, half) sums column slice
 // q of its half over all pairs (exact integer sums, in pair order) and runs
 // the epilogue on it.  For layers with too few tiles to occupy the GPU.
-template <int MODE, bool LR, bool ACT, bool SPLIT = false>
+template <int MODE, bool LR, bool ACT, int SPLIT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
@@ -259,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   static_assert(!SPLIT || (MODE == 1 && !LR), "split-K form: W4A4 without the low-rank branch");
   static_assert(!SPLIT || BM * kPartPitch <= C::kRing, "split-K partial inside the ring area");
+  static_assert(!SPLIT || kTOff + BM * (2 * 128 + 16) <= C::kRing, "split-K T rows (rank <= 128) in the ring area");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -860,12 +863,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pair order (exact int32), then the epilogue of the unsplit form.  A
       // thread keeps one group of four columns (their scales and bias in
       // registers) and walks rows `step` apart, two rows' loads in flight.
+      // With a low-rank branch (rank r = p.rank > 0) the slice's columns of
+      // L2 wait in the idle epilogue staging area as fp32 and its rows of T
+      // beside the partials, and each output adds sum_t T[m][t] L2[t][n]
+      // (fp32 fused multiply-adds, even and odd t in two chains) before the
+      // bias, like the persistent form's low-rank MMA does.
       const int S = prm.split;
-      const int per_row = BN / S / 4;                    // column groups in the slice
+      const int cw = BN / S;                             // columns in the slice
+      const int per_row = cw / 4;                        // column groups in the slice
       const int step = 16 * 32 / per_row;                // rows per pass
-      const int c = (int)(crank >> 1) * (BN / S) + (threadIdx.x % per_row) * 4;
+      const int cs = (threadIdx.x % per_row) * 4;        // this thread's columns within the slice
+      const int c = (int)(crank >> 1) * cw + cs;
       const int n = tile_n(0) + c;
       const int row0 = threadIdx.x / per_row;
+      const int lr_rank = SPLIT == 2 ? p.rank : 0;
+      const uint32_t l2s = sbase + (uint32_t)C::kOutOff;  // fp32 L2 slice [r][cw]
+      const uint32_t ts = sbase + (uint32_t)kTOff;        // bf16 T rows [128][r], pitch 2r + 16
+      const int t_pitch = 2 * lr_rank + 16;
+      if (lr_rank > 0) {
+        // every load of both tiles in flight at once, then one barrier
+        const int n_lo = tile_n(0) + (int)(crank >> 1) * cw;
+        for (int i = threadIdx.x; i < lr_rank * per_row; i += 16 * 32) {
+          const int t = i / per_row, v = i - t * per_row;
+          uint2 h = make_uint2(0u, 0u);
+          if (n_lo + 4 * v < p.N) h = __ldg(reinterpret_cast<const uint2*>(p.L2 + (long)t * p.N + n_lo + 4 * v));
+          st_shared_v4(l2s + (uint32_t)((t * cw + 4 * v) * 4),
+                       make_uint4(h.x << 16, h.x & 0xFFFF0000u, h.y << 16, h.y & 0xFFFF0000u));
+        }
+        const int t_vecs = lr_rank / 8;                   // 16-byte vectors per T row
+        for (int i = threadIdx.x; i < BM * t_vecs; i += 16 * 32) {
+          const int row = i / t_vecs, v = i - row * t_vecs;
+          const long m = (long)tile_m(0) + row;
+          uint4 tv = make_uint4(0u, 0u, 0u, 0u);
+          if (m < p.M) tv = __ldg(reinterpret_cast<const uint4*>(p.T + m * (long)lr_rank + 8 * v));
+          st_shared_v4(ts + (uint32_t)(row * t_pitch + 16 * v), tv);
+        }
+        named_barrier_sync(1, 16 * 32);
+      }
       if (n < p.N) {
         float sw[4], bv[4];
 #pragma unroll
@@ -907,8 +941,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (uint32_t)((int)acc[2] >> kShift), (uint32_t)((int)acc[3] >> kShift));
             float y[4];
 #pragma unroll
+            for (int j = 0; j < 4; ++j) y[j] = __fmul_rn(__fmul_rn(acc_to_float<true>(acc[j]), sa[k]), sw[j]);
+            if (lr_rank > 0) {
+              // plain shared-memory reads, so that the compiler batches the
+              // eight L2 rows of a step ahead of the multiply-adds; even and
+              // odd ranks accumulate separately and meet at the end
+              const float4* l2p = reinterpret_cast<const float4*>(smem_raw + (l2s - raw)) + cs / 4;
+              const uint4* tp = reinterpret_cast<const uint4*>(smem_raw + (ts - raw) + row * t_pitch);
+              float2 e01 = make_float2(0.0f, 0.0f), e23 = e01, o01 = e01, o23 = e01;
+              for (int t0 = 0; t0 < lr_rank; t0 += 8) {
+                const uint4 tv = tp[t0 / 8];
+                float4 lv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) lv[u] = l2p[(t0 + u) * (cw / 4)];
+                const uint32_t tw[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                for (int u = 0; u < 8; u += 2) {
+                  const float te = __uint_as_float(tw[u / 2] << 16);
+                  const float to = __uint_as_float(tw[u / 2] & 0xFFFF0000u);
+                  e01 = __ffma2_rn(make_float2(te, te), make_float2(lv[u].x, lv[u].y), e01);
+                  e23 = __ffma2_rn(make_float2(te, te), make_float2(lv[u].z, lv[u].w), e23);
+                  o01 = __ffma2_rn(make_float2(to, to), make_float2(lv[u + 1].x, lv[u + 1].y), o01);
+                  o23 = __ffma2_rn(make_float2(to, to), make_float2(lv[u + 1].z, lv[u + 1].w), o23);
+                }
+              }
+              const float2 l01 = __fadd2_rn(e01, o01), l23 = __fadd2_rn(e23, o23);
+              y[0] = __fadd_rn(y[0], l01.x);
+              y[1] = __fadd_rn(y[1], l01.y);
+              y[2] = __fadd_rn(y[2], l23.x);
+              y[3] = __fadd_rn(y[3], l23.y);
+            }
+#pragma unroll
             for (int j = 0; j < 4; ++j) {
-              y[j] = __fadd_rn(__fmul_rn(__fmul_rn(acc_to_float<true>(acc[j]), sa[k]), sw[j]), bv[j]);
+              y[j] = __fadd_rn(y[j], bv[j]);
               if constexpr (ACT) y[j] = gelu_tanh(y[j]);
             }
             __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
@@ -930,7 +995,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 // split > 1 (SPLIT): one cluster of `split` pairs per tile, all resident at once.
-template <int MODE, bool LR, bool ACT = false, bool SPLIT = false>
+template <int MODE, bool LR, bool ACT = false, int SPLIT = 0>
 cudaError_t launch_impl(const GemmArgs& a, unsigned int* err, cudaStream_t st, int split = 1) {
   using C = Cfg<MODE, LR>;
   auto kern = gemm_kernel<MODE, LR, ACT, SPLIT>;
@@ -996,11 +1061,13 @@ unsigned int* device_error_word();
 
 namespace {
 
-// K slices for the split-K form of a W4A4 layer without the low-rank branch:
-// 4 or 2 when the layer has too few 256 x 256 tiles to give every TPC one
-// (tiles x slices <= SMs / 2), each slice keeps at least two k-blocks, and
-// every cluster of 2 x slices CTAs fits on the GPU at once; else 1 (the
-// persistent form).
+// K slices for the split-K form of a W4A4 layer: 4 or 2 when the layer has
+// too few 256 x 256 tiles to give every TPC one (tiles x slices <= SMs / 2),
+// each slice keeps at least two k-blocks, a low-rank branch is small (rank
+// <= 32) on a long K range (>= 48 k-blocks) with its fp32 slice of L2 within
+// the 32 KB epilogue staging area, and every
+// cluster of 2 x slices CTAs fits on the GPU at once; else 1 (the persistent
+// form).
 struct SplitKey {
   int64_t v[4];
 };
@@ -1014,13 +1081,17 @@ cudaError_t plan_split(const GemmArgs& a, int* split) {
   const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + 255) / 256);
   const int nkb = a.K / BK;
   static PlanCache<SplitKey, int, 32> cache;
-  const SplitKey key = {{dev, tiles, nkb, sms}};
+  const SplitKey key = {{dev, tiles, nkb, sms + ((int64_t)a.rank << 32)}};
   const bool ok = cache.get(key, *split, [&](int& out) {
     out = 1;
     using C = Cfg<1, false>;
-    auto kern = gemm_kernel<1, false, ACT, true>;
+    auto kern = gemm_kernel<1, false, ACT, 1>;
     for (int s : {4, 2}) {
-      if (tiles * s > sms / 2 || nkb < 2 * s) continue;
+      if (tiles * s > sms / 2 || nkb < 2 * s || a.rank * (256 / s) * 4 > kOutStageBytes) continue;
+      // the low-rank term runs on CUDA cores here (M N r fused multiply-adds,
+      // ~0.13 us per unit of rank at M = 256, N = 3072): worth it only for a
+      // small rank on a long K range
+      if (a.rank > 32 || (a.rank > 0 && nkb < 48)) continue;
       if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes)) !=
           cudaSuccess)
         return false;
@@ -1054,13 +1125,16 @@ cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st) {
   if (!err) return cudaErrorInvalidDevicePointer;
   if (mode == GemmMode::kW8A8) return launch_impl<0, false>(a, err, st);
   if (mode == GemmMode::kW4A8) return launch_impl<2, false>(a, err, st);
-  if (a.rank == 0) {
+  {
     int split = 1;
     cudaError_t e = a.act == 1 ? plan_split<true>(a, &split) : plan_split<false>(a, &split);
     if (e != cudaSuccess) return e;
+    if (split > 1 && a.rank > 0)
+      return a.act == 1 ? launch_impl<1, false, true, 2>(a, err, st, split)
+                        : launch_impl<1, false, false, 2>(a, err, st, split);
     if (split > 1)
-      return a.act == 1 ? launch_impl<1, false, true, true>(a, err, st, split)
-                        : launch_impl<1, false, false, true>(a, err, st, split);
+      return a.act == 1 ? launch_impl<1, false, true, 1>(a, err, st, split)
+                        : launch_impl<1, false, false, 1>(a, err, st, split);
   }
   if (a.act == 1)
     return a.rank > 0 ? launch_impl<1, true, true>(a, err, st) : launch_impl<1, false, true>(a, err, st);

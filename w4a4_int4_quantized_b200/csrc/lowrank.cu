@@ -6,9 +6,10 @@
 // fp32 and is stored as bf16 for the up-projection folded into the GEMM.
 //
 // A thin product (N = rank <= 256), so the kernel splits K over a cluster of
-// S CTAs (2 <= S <= 8, any size) to put enough SMs on the activations: each CTA streams a
-// 128-row tile of X (K-major, 128-byte swizzle) and the matching rows of L1
-// (N-major, 128-byte swizzle) through a 4- to 8-deep TMA ring and accumulates its K
+// S CTAs (2 <= S <= 16, any size; above 8 a non-portable cluster size) to
+// put enough SMs on the activations: each CTA streams a 128-row tile of X
+// (K-major, 128-byte swizzle) and the matching rows of L1 (N-major, 128-byte
+// swizzle) through a 4- to 8-deep TMA ring and accumulates its K
 // slice with tcgen05.mma kind::f16 into TMEM.  The fp32 partials are drained
 // into each CTA's shared memory and reduced through distributed shared memory
 // in a fixed CTA order (deterministic, no global scratch); CTA c writes rows
@@ -31,6 +32,7 @@ namespace {
 constexpr int BM = 128;        // rows of X per tile
 constexpr int BKL = 64;        // K per stage (128 bytes of bf16: one swizzle row)
 constexpr int NSTMAX = 8;      // TMA stages (as many as fit: 4 to 8)
+constexpr int kMaxSplit = 16;  // K split (cluster size): 16 needs the non-portable cluster size
 constexpr int kThreads = 128;
 
 struct LrBarriers {
@@ -48,6 +50,9 @@ struct LrParams {
   int withhold;                 // self-test: the producer issues no operand load
 };
 
+// MAXS: the largest split S this instantiation reduces (8 or 16; the
+// reduction loop is unrolled to it).
+template <int MAXS>
 __global__ void __launch_bounds__(kThreads, 1)
     lowrank_down_kernel(const LrParams p, const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmL1) {
@@ -176,13 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rr = row0 + item / vec_per_row;
     const int c = (item % vec_per_row) * 4;
     const uint32_t local = sbase + (uint32_t)(rr * part_pitch + c * 4);
-    uint4 w[8];
+    uint4 w[MAXS];
 #pragma unroll
-    for (int s = 0; s < 8; ++s)
+    for (int s = 0; s < MAXS; ++s)
       if (s < S) w[s] = ld_cluster_v4(map_to_rank(local, (uint32_t)s));
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+    for (int s = 0; s < MAXS; ++s) {
       if (s < S) {
         acc[0] = __fadd_rn(acc[0], __uint_as_float(w[s].x));
         acc[1] = __fadd_rn(acc[1], __uint_as_float(w[s].y));
@@ -227,11 +232,14 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   const int smem = data + (int)sizeof(LrBarriers) + 1024;
   static DeviceFlags attr_set;
   if (!attr_set.done(dev)) {
-    e = cudaFuncSetAttribute(lowrank_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
-    if (e != cudaSuccess) return e;
+    for (auto k : {lowrank_down_kernel<8>, lowrank_down_kernel<kMaxSplit>}) {
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448)) != cudaSuccess ||
+          (e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+        return e;
+    }
     attr_set.set(dev);
   }
-  // K split S (cluster size): the largest S <= 8 for which every cluster of
+  // K split S (cluster size): the largest S <= 16 for which every cluster of
   // the grid is resident at once.  Clusters must fit inside one GPC, so the
   // count that fits is below sms / S for the larger S; a grid past it runs a
   // second wave and doubles the time.
@@ -243,7 +251,7 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   int S = 1;
   const bool ok = split_cache.get(key, S, [&](int& out) {
     out = 1;
-    for (int sc = std::min(8, nkb); sc >= 2 && out == 1; --sc) {
+    for (int sc = std::min(kMaxSplit, nkb); sc >= 2 && out == 1; --sc) {
       if (m_tiles * sc > sms) continue;
       cudaLaunchConfig_t qc = {};
       qc.gridDim = dim3(m_tiles * sc, 1, 1);
@@ -257,7 +265,9 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
       qc.attrs = &qa;
       qc.numAttrs = 1;
       int max_clusters = 0;
-      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, lowrank_down_kernel, &qc)) != cudaSuccess) return false;
+      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, sc > 8 ? lowrank_down_kernel<kMaxSplit> : lowrank_down_kernel<8>,
+                                               &qc)) != cudaSuccess)
+        return false;
       if (m_tiles <= max_clusters) out = sc;
     }
     return true;
@@ -284,7 +294,8 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   LrParams prm{T, M, K, r, S, nst, err, wait_ns, withhold};
-  e = cudaLaunchKernelEx(&cfg, lowrank_down_kernel, prm, tX, tL1);
+  e = S > 8 ? cudaLaunchKernelEx(&cfg, lowrank_down_kernel<kMaxSplit>, prm, tX, tL1)
+            : cudaLaunchKernelEx(&cfg, lowrank_down_kernel<8>, prm, tX, tL1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
