@@ -311,6 +311,20 @@ def test_split_k_equals_the_persistent_form(K, act):
     assert torch.equal(Y_few.view(torch.int16), Y_all[:256].view(torch.int16))
 
 
+def test_split_k_w4a8_equals_the_persistent_form():
+    """The W4A8 GEMM's split-K form: the first 256 rows of a 4608-row layer
+    bit for bit the same as those rows run on their own."""
+    import torch
+    M, N, K, g = 4608, 3072, 12288, 128
+    d = _layer(M, N, K, g, 0, True, seed=77)
+    X, W, b = dev_bf16(d["X"]), dev_bf16(d["W"]), dev_bf16(d["bias"])
+    Wq, ws, wz = w4.w4a8_quantize_weights(W, g)
+    Y_all = w4.w4a8_linear(X, Wq, ws, wz, g, b)
+    Y_few = w4.w4a8_linear(X[:256].contiguous(), Wq, ws, wz, g, b)
+    torch.cuda.synchronize()
+    assert torch.equal(Y_few.view(torch.int16), Y_all[:256].view(torch.int16))
+
+
 def test_fused_mlp_chain():
     """w4a4_mlp = down(gelu(up(X))): its activated tensor is the fused
     up-projection (checked against the fp64 oracle), and its output equals the

@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   Barriers* bar = reinterpret_cast<Barriers*>(smem_raw + (sbase - raw) + C::kDataBytes);
 
-  static_assert(!SPLIT || (MODE == 1 && !LR), "split-K form: W4A4 without the low-rank branch");
+  static_assert(!SPLIT || (MODE != 0 && !LR && (SPLIT == 1 || MODE == 1)),
+                "split-K form: W4A4 (with the low-rank term in the reduction) or W4A8");
   static_assert(!SPLIT || BM * kPartPitch <= C::kRing, "split-K partial inside the ring area");
   static_assert(!SPLIT || kTOff + BM * (2 * 128 + 16) <= C::kRing, "split-K T rows (rank <= 128) in the ring area");
   const int warp = threadIdx.x >> 5;
@@ -941,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (uint32_t)((int)acc[2] >> kShift), (uint32_t)((int)acc[3] >> kShift));
             float y[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) y[j] = __fmul_rn(__fmul_rn(acc_to_float<true>(acc[j]), sa[k]), sw[j]);
+            for (int j = 0; j < 4; ++j) y[j] = __fmul_rn(__fmul_rn(acc_to_float<MODE == 1>(acc[j]), sa[k]), sw[j]);
             if (lr_rank > 0) {
               // plain shared-memory reads, so that the compiler batches the
               // eight L2 rows of a step ahead of the multiply-adds; even and
@@ -1061,17 +1062,16 @@ unsigned int* device_error_word();
 
 namespace {
 
-// K slices for the split-K form of a W4A4 layer: 4 or 2 when the layer has
+// K slices for the split-K form of a W4A4 or W4A8 layer: 4 or 2 when it has
 // too few 256 x 256 tiles to give every TPC one (tiles x slices <= SMs / 2),
 // each slice keeps at least two k-blocks, a low-rank branch is small (rank
 // <= 32) on a long K range (>= 48 k-blocks) with its fp32 slice of L2 within
-// the 32 KB epilogue staging area, and every
-// cluster of 2 x slices CTAs fits on the GPU at once; else 1 (the persistent
-// form).
+// the 32 KB epilogue staging area, and every cluster of 2 x slices CTAs fits
+// on the GPU at once; else 1 (the persistent form).
 struct SplitKey {
   int64_t v[4];
 };
-template <bool ACT>
+template <int MODE, bool ACT>
 cudaError_t plan_split(const GemmArgs& a, int* split) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1084,8 +1084,8 @@ cudaError_t plan_split(const GemmArgs& a, int* split) {
   const SplitKey key = {{dev, tiles, nkb, sms + ((int64_t)a.rank << 32)}};
   const bool ok = cache.get(key, *split, [&](int& out) {
     out = 1;
-    using C = Cfg<1, false>;
-    auto kern = gemm_kernel<1, false, ACT, 1>;
+    using C = Cfg<MODE, false>;
+    auto kern = gemm_kernel<MODE, false, ACT, 1>;
     for (int s : {4, 2}) {
       if (tiles * s > sms / 2 || nkb < 2 * s || a.rank * (256 / s) * 4 > kOutStageBytes) continue;
       // the low-rank term runs on CUDA cores here (M N r fused multiply-adds,
@@ -1124,10 +1124,15 @@ cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st) {
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorInvalidDevicePointer;
   if (mode == GemmMode::kW8A8) return launch_impl<0, false>(a, err, st);
-  if (mode == GemmMode::kW4A8) return launch_impl<2, false>(a, err, st);
+  if (mode == GemmMode::kW4A8) {
+    int split = 1;
+    cudaError_t e = plan_split<2, false>(a, &split);
+    if (e != cudaSuccess) return e;
+    return split > 1 ? launch_impl<2, false, false, 1>(a, err, st, split) : launch_impl<2, false>(a, err, st);
+  }
   {
     int split = 1;
-    cudaError_t e = a.act == 1 ? plan_split<true>(a, &split) : plan_split<false>(a, &split);
+    cudaError_t e = a.act == 1 ? plan_split<1, true>(a, &split) : plan_split<1, false>(a, &split);
     if (e != cudaSuccess) return e;
     if (split > 1 && a.rank > 0)
       return a.act == 1 ? launch_impl<1, false, true, 2>(a, err, st, split)
