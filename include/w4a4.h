@@ -296,6 +296,20 @@ w4a4_status w4a4_bake_lora_sr(const void* W, const void* A, const void* B, int l
 w4a4_status w4a4_plan_rotate_quantize(int M, int K, int group, int sms, int resident_per_sm, int cached,
                                       int* shape);
 
+/* Host-only view of the GEMM's split-K decision (w4a4_gemm, w4a4_gemm_gelu
+ * and w4a8_gemm, and the layers built on them): no CUDA call.  A layer whose
+ * 256 x 256 output tiles are too few to give every pair of SMs one runs with
+ * its K range split over a cluster of 2 x *split CTAs per tile, the int32
+ * partials summed exactly through distributed shared memory.  Given M, N, K
+ * (shape rules as w4a4_gemm with group 128), the low-rank rank (0 .. 256, a
+ * multiple of 16), a device with `sms` SMs on which `clusters_of_8` clusters
+ * of 8 CTAs and `clusters_of_4` of 4 (one CTA per SM) fit at once, writes
+ * *split = 4, 2, or 1 for the persistent form.  The launchers make the same
+ * decision with the device's own occupancy figures.  The pages have no
+ * counterpart. */
+w4a4_status w4a4_plan_gemm_split(int M, int N, int K, int rank, int sms, int clusters_of_8, int clusters_of_4,
+                                 int* split);
+
 /* ---------------------------------------------------------------- failures */
 /* Kernels never trap: a wait on another part of the kernel that runs past its
  * time limit (2 s) records a code in a per-device error word and lets the

@@ -264,3 +264,36 @@ def test_launch_plan_cache_under_host_threads(lib):
 
     with cf.ThreadPoolExecutor(8) as ex:
         assert sum(ex.map(worker, range(8))) == 0
+
+
+@pytest.mark.parametrize("M,N,K,rank,kw,expect", [
+    (256, 3072, 3072, 0, {}, 4),          # 12 tiles: four pairs per tile fill 48 of 74 pairs
+    (512, 3072, 3072, 0, {}, 2),          # 24 tiles: 4 x 24 > 74, 2 x 24 fits
+    (4608, 3072, 3072, 0, {}, 1),         # 216 tiles: the persistent form
+    (40, 8, 3072, 0, {}, 4),              # one tile
+    (64, 256, 256, 0, {}, 1),             # two k-blocks: no slice would keep two
+    (1, 3072, 512, 0, {}, 2),             # four k-blocks: two slices of two
+    (256, 3072, 12288, 16, {}, 4),        # small rank on a long K range
+    (256, 3072, 12288, 32, {}, 4),
+    (256, 3072, 12288, 64, {}, 1),        # larger ranks keep the tensor-core low-rank MMA
+    (256, 3072, 3072, 16, {}, 1),         # short K range with a low-rank branch
+    (256, 3072, 3072, 0, {"clusters_of_8": 8}, 2),                      # 12 clusters of 8 do not fit
+    (256, 3072, 3072, 0, {"clusters_of_8": 8, "clusters_of_4": 8}, 1),  # nor 12 of 4
+    (256, 3072, 3072, 0, {"sms": 40}, 1),                               # too few SMs for any split
+])
+def test_plan_gemm_split(M, N, K, rank, kw, expect):
+    """The GEMM's split-K decision, host only: the same function the
+    launchers call with the device's occupancy figures."""
+    assert w4.w4a4_plan_gemm_split(M, N, K, rank, **kw) == expect
+
+
+def test_plan_gemm_split_validation(lib):
+    import ctypes
+    out = ctypes.c_int(0)
+    f = lib.w4a4_plan_gemm_split
+    assert f(256, 3072, 3072, 0, 148, 16, 32, None) == 1                  # W4A4_ERR_INVALID_ARG
+    assert f(256, 3070, 3072, 0, 148, 16, 32, ctypes.byref(out)) == 2     # N not a multiple of 8
+    assert f(256, 3072, 3000, 0, 148, 16, 32, ctypes.byref(out)) == 2     # K not a multiple of 128
+    assert f(256, 3072, 3072, 20, 148, 16, 32, ctypes.byref(out)) == 2    # rank not a multiple of 16
+    assert f(0, 3072, 3072, 0, 148, 16, 32, ctypes.byref(out)) == 2       # empty M
+    assert f(256, 3072, 3072, 0, 148, 16, 32, ctypes.byref(out)) == 0 and out.value == 4

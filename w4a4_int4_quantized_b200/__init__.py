@@ -24,6 +24,7 @@ __all__ = [
     "w8a8_workspace_bytes", "w4a8_quantize_weights", "w4a8_gemm", "w4a8_linear", "w4a8_workspace_bytes",
     "w4a4_lora_merge", "w4a4_gemm_gelu", "w4a4_linear_gelu", "w4a4_mlp", "w4a4_mlp_workspace_bytes",
     "w4a4_bake_lora_sr", "w4a4_get_device_error", "w4a4_selftest_wait_timeout", "w4a4_plan_rotate_quantize",
+    "w4a4_plan_gemm_split",
     "DEVERR_WAIT_OPERANDS", "DEVERR_WAIT_SLOT", "DEVERR_WAIT_ACCUM", "DEVERR_WAIT_DRAIN",
 ]
 
@@ -87,6 +88,7 @@ def load_library():
         "w4a4_get_device_error": ([P, ctypes.POINTER(ctypes.c_uint)], S),
         "w4a4_selftest_wait_timeout": ([P, P, I, I, I, P, ctypes.c_uint, P], S),
         "w4a4_plan_rotate_quantize": ([I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)], S),
+        "w4a4_plan_gemm_split": ([I, I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)], S),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -407,3 +409,13 @@ def w4a4_plan_rotate_quantize(M, K, group, sms=148, resident_per_sm=4, cached=Tr
     _check("w4a4_plan_rotate_quantize", load_library().w4a4_plan_rotate_quantize(
         M, K, group, sms, resident_per_sm, 1 if cached else 0, out))
     return tuple(out)
+
+
+def w4a4_plan_gemm_split(M, N, K, rank=0, sms=148, clusters_of_8=16, clusters_of_4=32):
+    """K slices the GEMM would split a layer over (4 or 2; 1 = the persistent
+    form), for a device with `sms` SMs on which the given numbers of 8- and
+    4-CTA clusters fit at once (host only, no CUDA call)."""
+    out = ctypes.c_int(0)
+    _check("w4a4_plan_gemm_split", load_library().w4a4_plan_gemm_split(
+        M, N, K, rank, sms, clusters_of_8, clusters_of_4, ctypes.byref(out)))
+    return out.value

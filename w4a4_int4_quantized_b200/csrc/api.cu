@@ -386,6 +386,18 @@ w4a4_status w4a4_plan_rotate_quantize(int M, int K, int group, int sms, int resi
                                                                                            : W4A4_ERR_UNSUPPORTED_SHAPE;
 }
 
+w4a4_status w4a4_plan_gemm_split(int M, int N, int K, int rank, int sms, int clusters_of_8, int clusters_of_4,
+                                  int* split) {
+  if (!split) return W4A4_ERR_INVALID_ARG;
+  if (M < 1 || N < 8 || N % 8 != 0 || sms < 2 || clusters_of_8 < 0 || clusters_of_4 < 0)
+    return W4A4_ERR_UNSUPPORTED_SHAPE;
+  w4a4_status s = check_rank(rank);
+  if (s != W4A4_OK) return s;
+  if ((s = check_k_group(K, 128)) != W4A4_OK) return s;
+  return plan_gemm_split(M, N, K, rank, sms, clusters_of_8, clusters_of_4, split) ? W4A4_OK
+                                                                                  : W4A4_ERR_UNSUPPORTED_SHAPE;
+}
+
 // ------------------------------------------------------------------ failures
 w4a4_status w4a4_selftest_wait_timeout(const void* X, const void* L1, int M, int K, int rank, void* T,
                                        unsigned int timeout_us, w4a4_stream_t stream) {

@@ -1071,6 +1071,27 @@ namespace {
 struct SplitKey {
   int64_t v[4];
 };
+
+// The decision itself, a pure host function: `resident(s, clusters)` gives
+// how many clusters of 2 s CTAs (one per SM) fit on the GPU at once.
+template <class Resident>
+bool choose_split(int tiles, int nkb, int rank, int sms, Resident&& resident, int& out) {
+  out = 1;
+  for (int s : {4, 2}) {
+    if (tiles * s > sms / 2 || nkb < 2 * s || rank * (256 / s) * 4 > kOutStageBytes) continue;
+    // the low-rank term runs on CUDA cores here (M N r fused multiply-adds,
+    // ~0.13 us per unit of rank at M = 256, N = 3072): worth it only for a
+    // small rank on a long K range
+    if (rank > 32 || (rank > 0 && nkb < 48)) continue;
+    int clusters = 0;
+    if (!resident(s, clusters)) return false;
+    if (clusters >= tiles) {
+      out = s;
+      break;
+    }
+  }
+  return true;
+}
 template <int MODE, bool ACT>
 cudaError_t plan_split(const GemmArgs& a, int* split) {
   int dev = 0;
@@ -1083,15 +1104,9 @@ cudaError_t plan_split(const GemmArgs& a, int* split) {
   static PlanCache<SplitKey, int, 32> cache;
   const SplitKey key = {{dev, tiles, nkb, sms + ((int64_t)a.rank << 32)}};
   const bool ok = cache.get(key, *split, [&](int& out) {
-    out = 1;
     using C = Cfg<MODE, false>;
     auto kern = gemm_kernel<MODE, false, ACT, 1>;
-    for (int s : {4, 2}) {
-      if (tiles * s > sms / 2 || nkb < 2 * s || a.rank * (256 / s) * 4 > kOutStageBytes) continue;
-      // the low-rank term runs on CUDA cores here (M N r fused multiply-adds,
-      // ~0.13 us per unit of rank at M = 256, N = 3072): worth it only for a
-      // small rank on a long K range
-      if (a.rank > 32 || (a.rank > 0 && nkb < 48)) continue;
+    return choose_split(tiles, nkb, a.rank, sms, [&](int s, int& clusters) {
       if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes)) !=
           cudaSuccess)
         return false;
@@ -1106,19 +1121,21 @@ cudaError_t plan_split(const GemmArgs& a, int* split) {
       qa.val.clusterDim.z = 1;
       qc.attrs = &qa;
       qc.numAttrs = 1;
-      int clusters = 0;
-      if ((e = cudaOccupancyMaxActiveClusters(&clusters, kern, &qc)) != cudaSuccess) return false;
-      if (clusters >= tiles) {
-        out = s;
-        break;
-      }
-    }
-    return true;
+      return (e = cudaOccupancyMaxActiveClusters(&clusters, kern, &qc)) == cudaSuccess;
+    }, out);
   });
   return ok ? cudaSuccess : e;
 }
 
 }  // namespace
+
+bool plan_gemm_split(int M, int N, int K, int rank, int sms, int clusters_of_8, int clusters_of_4, int* split) {
+  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
+  return choose_split(tiles, K / BK, rank, sms, [&](int s, int& clusters) {
+    clusters = s == 4 ? clusters_of_8 : clusters_of_4;
+    return true;
+  }, *split);
+}
 
 cudaError_t launch_gemm(const GemmArgs& a, GemmMode mode, cudaStream_t st) {
   unsigned int* err = device_error_word();

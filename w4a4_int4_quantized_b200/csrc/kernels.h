@@ -15,6 +15,11 @@ cudaError_t launch_rotate_quantize(const uint16_t* X, int rows, int K, int group
 // out = {rows per block, threads, dynamic shared memory, grid}.
 bool plan_rotate_quantize_shape(int M, int K, int group, int sms, int resident_per_sm, bool cached, int out[4]);
 
+// The GEMM's split-K decision without a CUDA call (the launcher feeds it the
+// occupancy query): *split = 4, 2 or 1 (the persistent form), given how many
+// clusters of 8 and of 4 CTAs fit on the device at once.
+bool plan_gemm_split(int M, int N, int K, int rank, int sms, int clusters_of_8, int clusters_of_4, int* split);
+
 struct GemmArgs {
   const uint8_t* A;        // activation codes [M, K/2] packed or [M, K] int8
   const float* a_scale;    // [M]
