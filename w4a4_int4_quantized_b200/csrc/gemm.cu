@@ -135,6 +135,11 @@ struct Cfg {
   // order, so a phase-parity wait can never match a fill two phases old
   static_assert(PS % kSets == 0, "each widen set owns its packed stages");
   static_assert(US >= kSets && kLead >= 1, "widened ring");
+  // W4A8: the kLead k-blocks widened ahead of an epilogue also need their
+  // int8 A tiles; slot g + kLead - 1 frees only once the MMAs have read
+  // k-block g + kLead - 1 - AS, which must belong to the finished tile (else
+  // the epilogue, the MMAs and the A loads wait on one another)
+  static_assert(MODE != 2 || kLead <= AS, "W4A8: A ring deeper than the k-blocks widened ahead");
   static_assert(kWOff % 1024 == 0 && kAOff % 1024 == 0, "128-byte swizzle atoms");
   static_assert(kWOff + US * kWideB <= kRing && (MODE != 2 || kAOff + AS * kI8A <= kRing), "rings inside the ring area");
   static_assert(!LR || MODE == 1, "low-rank branch: W4A4 only");
