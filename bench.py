@@ -52,8 +52,8 @@ def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
 # they were taken from (sha256 prefix); reported as null once the source
 # changes.
 MEASURED_TRAFFIC = {
-    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6cf834b8706ed0d0", 11.883e6),
-    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "6cf834b8706ed0d0", 20.498e6),
+    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "14dc41e744ee55af", 11.890e6),
+    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "14dc41e744ee55af", 20.498e6),
     ("rotate_quantize", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/quantize.cu", "59bbaf52c3e58355", 28.378e6),
 }
 
