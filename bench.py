@@ -48,24 +48,33 @@ def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
     return 2.0 * INT8_MAC_PER_CLK_PER_SM * sms * sm_mhz * 1e6 / 1e12
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# the ncu captures summarised in profiles/, valid only for the kernel source
-# they were taken from (sha256 prefix); reported as null once the source
-# changes.
+# the ncu captures summarised in profiles/, valid only for the kernel code they
+# were taken from: keyed by a hash of the source file with its comments and
+# whitespace removed (so an edited comment keeps the figure, any code change
+# drops it to null).
 MEASURED_TRAFFIC = {
-    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "14dc41e744ee55af", 11.890e6),
-    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "14dc41e744ee55af", 20.498e6),
-    ("rotate_quantize", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/quantize.cu", "59bbaf52c3e58355", 28.378e6),
+    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "7763607990f1ad98", 11.890e6),
+    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "7763607990f1ad98", 20.498e6),
+    ("rotate_quantize", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/quantize.cu", "003946100a4d56c2", 28.378e6),
 }
+
+
+def code_hash(text: str) -> str:
+    """sha256 prefix of C/C++/CUDA source with comments and whitespace removed."""
+    import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()[:16]
 
 
 def _traffic(kernel: str, workload: str):
     if (kernel, workload) not in MEASURED_TRAFFIC:
         return None
-    import hashlib
     path, sha, value = MEASURED_TRAFFIC[(kernel, workload)]
     try:
-        with open(os.path.join(ROOT, path), "rb") as f:
-            cur = hashlib.sha256(f.read()).hexdigest()[:16]
+        with open(os.path.join(ROOT, path)) as f:
+            cur = code_hash(f.read())
     except OSError:
         return None
     return value if cur == sha else None

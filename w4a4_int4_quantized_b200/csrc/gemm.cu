@@ -45,7 +45,8 @@
 //               stores.
 // The kernel is persistent: one pair per TPC walks its output tiles, and the
 // TMA and widen stages run ahead into the next tile while the epilogue of the
-// current one drains the accumulator.  With a low-rank branch the tile stays
+// current one drains the accumulator (layers with too few tiles use the
+// split-K form described at the kernel instead).  With a low-rank branch the tile stays
 // 256 x 256 and TMEM holds no second accumulator: the epilogue rewrites the
 // int32 accumulator in place as fp32 (acc s_a) s_w', bf16 MMAs accumulate
 // T L2 onto it (operand chunks of 128 ranks staged by TMA), and a second read
@@ -239,13 +240,13 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return 0.5f * x * (1.0f + tanhf(u));
 }
 
-// SPLIT 1 (W4A4) or 2 (W4A4 with a small low-rank branch, its term added in
-// the reduction): a cluster of prm.split pairs shares one 256 x 256 tile;
-// pair q accumulates the k-blocks
-// [q nk / split, (q + 1) nk / split), every CTA leaves its int32 partial in
-// shared memory, and after a cluster barrier CTA (q, half) sums column slice
-// q of its half over all pairs (exact integer sums, in pair order) and runs
-// the epilogue on it.  For layers with too few tiles to occupy the GPU.
+// SPLIT 1 (W4A4 or W4A8) or 2 (W4A4 with a small low-rank branch, its term
+// added in the reduction): a cluster of prm.split pairs shares one 256 x 256
+// tile; pair q accumulates the k-blocks [q nk / split, (q + 1) nk / split),
+// every CTA leaves its int32 partial in shared memory, and after a cluster
+// barrier CTA (q, half) sums column slice q of its half over all pairs
+// (exact integer sums, in pair order) and runs the epilogue on it.  For
+// layers with too few tiles to occupy the GPU.
 template <int MODE, bool LR, bool ACT, int SPLIT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const Params prm, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
