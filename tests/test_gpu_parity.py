@@ -269,7 +269,8 @@ def test_w4a4_layer_with_runtime_lora(M, N, K, g, r, rl, scale):
     check_output(host_f64(Y), ref["Y"], lowrank=True)
 
 
-@pytest.mark.parametrize("M,N,K,g,r", [(130, 520, 1280, 64, 32), (257, 768, 3072, 128, 0)])
+@pytest.mark.parametrize("M,N,K,g,r", [(130, 520, 1280, 64, 32), (257, 768, 3072, 128, 0),
+                                     (256, 1024, 12288, 128, 32)])   # split-K, low-rank term in the reduction
 def test_w4a4_layer_with_fused_gelu(M, N, K, g, r):
     """GELU(tanh) fused into the epilogue: the same accumulators, GELU of the
     unrounded output within the layer tolerance, and the fused call equal to
