@@ -134,6 +134,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+// Asynchronous 16-byte copy from global to shared memory (cp.async); with
+// src_bytes < 16 the rest of the 16 bytes is zero-filled (0: nothing is read).
+// The issuing thread waits for its own copies with cp_async_wait_all; a
+// barrier after that wait publishes them to the other threads.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -88,7 +88,11 @@ constexpr int kStageTile = 32 * 32 * 2;            // epilogue staging tile: 32 
 constexpr int kOutStageBytes = 16 * kStageTile;    // one per epilogue warp
 constexpr int kBarBytes = 512;
 constexpr int kPartPitch = 256 * 4 + 16;           // split-K: int32 partial row pitch (bank-spread)
-constexpr int kTOff = 128 * kPartPitch;            // split-K: T rows after the partials (ring area)
+constexpr int kL2fOff = 128 * kPartPitch;          // split-K: fp32 L2 slice after the partials (ring area)
+constexpr int kSplitMaxRank = 32;                  // split-K: largest low-rank term (CUDA cores, reduction)
+constexpr int kSplitTOff = 8192;                   // split-K: T rows after the bf16 L2 slice (staging area)
+constexpr int kSplitSwOff = BM * 4;                // split-K vector area: row scales, column scales, bias
+constexpr int kSplitBiasOff = kSplitSwOff + 128 * 4;
 
 // MODE 0: W8A8 (int8 x int8, TMA straight into the MMA layout); 1: W4A4
 // (packed INT4 x packed INT4, both widened, A into TMEM); 2: W4A8 (the int8
@@ -185,6 +189,11 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "memory");
   return v;
 }
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
 
 // 16 packed bytes (32 codes) -> 32 widened bytes (two 16-byte chunks).
 __device__ __forceinline__ void widen16(const uint4 p, uint4& c0, uint4& c1) {
@@ -268,7 +277,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(!SPLIT || (MODE != 0 && !LR && (SPLIT == 1 || MODE == 1)),
                 "split-K form: W4A4 (with the low-rank term in the reduction) or W4A8");
   static_assert(!SPLIT || BM * kPartPitch <= C::kRing, "split-K partial inside the ring area");
-  static_assert(!SPLIT || kTOff + BM * (2 * 128 + 16) <= C::kRing, "split-K T rows (rank <= 128) in the ring area");
+  // split-K operands of the reduction: the fp32 L2 slice (<= 32 ranks x 128
+  // columns) after the partials; the bf16 slice and T rows in the epilogue
+  // staging area, idle in this form; scales and bias in the vector area
+  static_assert(!SPLIT || kL2fOff + kSplitMaxRank * 128 * 4 <= C::kRing, "split-K fp32 L2 slice in the ring area");
+  static_assert(!SPLIT || (kSplitMaxRank * 128 * 2 <= kSplitTOff &&
+                           kSplitTOff + BM * (2 * kSplitMaxRank + 16) <= C::kOutBytes),
+                "split-K bf16 L2 slice and T rows in the staging area");
+  static_assert(!SPLIT || kSplitBiasOff + 128 * 2 <= C::kVecBytes, "split-K scales and bias in the vector area");
+  static_assert(!SPLIT || BM / 4 + 128 / 4 + 128 / 8 <= 16 * 32, "split-K: one vector copy per epilogue thread");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -817,6 +834,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if constexpr (SPLIT) {
+      // The reduction's operands go to shared memory by cp.async while the
+      // k-blocks run (one 16-byte copy per thread, two for the low-rank
+      // operands; zero fill past M or N), so that none of its global loads
+      // waits after the cluster barrier: this CTA's row scales, its column
+      // slice's scales and bias, and with a low-rank term the slice's L2
+      // columns (bf16) and this CTA's T rows.
+      if (my_tiles > 0) {
+        const int t = threadIdx.x;                      // 0 .. 511
+        const int cw = BN / prm.split;
+        const int m0 = tile_m(0);
+        const int n_lo = tile_n(0) + (int)(crank >> 1) * cw;
+        const uint32_t vs = sbase + (uint32_t)C::kVecOff;
+        if (t < BM / 4) {
+          const int m = m0 + 4 * t;
+          const int nv = min(max(p.M - m, 0), 4);
+          cp_async_16(vs + (uint32_t)(16 * t), nv > 0 ? p.a_scale + m : p.a_scale, (uint32_t)(4 * nv));
+        } else if (t < BM / 4 + cw / 4) {
+          const int c = t - BM / 4, n = n_lo + 4 * c;    // N % 8 == 0: a chunk is wholly in or out
+          cp_async_16(vs + (uint32_t)(kSplitSwOff + 16 * c), n < p.N ? p.b_scale + n : p.b_scale, n < p.N ? 16u : 0u);
+        } else if (t < BM / 4 + cw / 4 + cw / 8) {
+          const int c = t - BM / 4 - cw / 4, n = n_lo + 8 * c;
+          const bool in = p.bias && n < p.N;
+          cp_async_16(vs + (uint32_t)(kSplitBiasOff + 16 * c), in ? (const void*)(p.bias + n) : (const void*)p.b_scale,
+                      in ? 16u : 0u);
+        }
+        if (SPLIT == 2 && p.rank > 0) {
+          const int r = p.rank;
+          const int tv = r / 8;                           // 16-byte chunks of a T row
+          const uint32_t ts = sbase + (uint32_t)(C::kOutOff + kSplitTOff);
+          for (int i = t; i < BM * tv; i += 16 * 32) {
+            const int row = i / tv, v = i - row * tv;
+            const long m = (long)m0 + row;
+            const bool in = m < p.M;
+            cp_async_16(ts + (uint32_t)(row * (2 * r + 16) + 16 * v), in ? p.T + m * r + 8 * v : p.T, in ? 16u : 0u);
+          }
+          const int lv = cw / 8;                          // 16-byte chunks of an L2 slice row
+          const uint32_t l2b = sbase + (uint32_t)C::kOutOff;
+          for (int i = t; i < r * lv; i += 16 * 32) {
+            const int k = i / lv, v = i - k * lv;
+            const int n = n_lo + 8 * v;
+            const bool in = n < p.N;
+            cp_async_16(l2b + (uint32_t)((k * cw + 8 * v) * 2), in ? p.L2 + (long)k * p.N + n : p.L2, in ? 16u : 0u);
+          }
+        }
+      }
       // one tile: widen this pair's k-blocks, then leave this warp's share
       // of the int32 partial (32 rows x 64 columns) in the ring area, idle
       // once the accumulator is final (every MMA has read its stages)
@@ -838,6 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_shared_v4(prow + (uint32_t)((ch * 32 + 4 * q) * 4),
                          make_uint4(v[ch][4 * q], v[ch][4 * q + 1], v[ch][4 * q + 2], v[ch][4 * q + 3]));
       }
+      cp_async_wait_all();   // published to the other threads by the cluster barrier below
     } else if (!PACKED) {
       for (int i = 0; i < my_tiles; ++i) epilogue(i);
     } else {
@@ -884,26 +947,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = tile_n(0) + c;
       const int row0 = threadIdx.x / per_row;
       const int lr_rank = SPLIT == 2 ? p.rank : 0;
-      const uint32_t l2s = sbase + (uint32_t)C::kOutOff;  // fp32 L2 slice [r][cw]
-      const uint32_t ts = sbase + (uint32_t)kTOff;        // bf16 T rows [128][r], pitch 2r + 16
+      const uint32_t l2s = sbase + (uint32_t)kL2fOff;                 // fp32 L2 slice [r][cw]
+      const uint32_t ts = sbase + (uint32_t)(C::kOutOff + kSplitTOff);  // bf16 T rows [128][r], pitch 2r + 16
       const int t_pitch = 2 * lr_rank + 16;
+      const uint8_t* vec_b = smem_raw + (sbase - raw) + C::kVecOff;
+      const float* vec = reinterpret_cast<const float*>(vec_b);                        // row scales
+      const float* vec_sw = reinterpret_cast<const float*>(vec_b + kSplitSwOff);       // column scales
+      const uint16_t* vec_bias = reinterpret_cast<const uint16_t*>(vec_b + kSplitBiasOff);
       if (lr_rank > 0) {
-        // every load of both tiles in flight at once, then one barrier
-        const int n_lo = tile_n(0) + (int)(crank >> 1) * cw;
+        // the bf16 slice (loaded during the k-blocks) widened to fp32 once
+        const uint32_t l2b = sbase + (uint32_t)C::kOutOff;
         for (int i = threadIdx.x; i < lr_rank * per_row; i += 16 * 32) {
-          const int t = i / per_row, v = i - t * per_row;
-          uint2 h = make_uint2(0u, 0u);
-          if (n_lo + 4 * v < p.N) h = __ldg(reinterpret_cast<const uint2*>(p.L2 + (long)t * p.N + n_lo + 4 * v));
-          st_shared_v4(l2s + (uint32_t)((t * cw + 4 * v) * 4),
-                       make_uint4(h.x << 16, h.x & 0xFFFF0000u, h.y << 16, h.y & 0xFFFF0000u));
-        }
-        const int t_vecs = lr_rank / 8;                   // 16-byte vectors per T row
-        for (int i = threadIdx.x; i < BM * t_vecs; i += 16 * 32) {
-          const int row = i / t_vecs, v = i - row * t_vecs;
-          const long m = (long)tile_m(0) + row;
-          uint4 tv = make_uint4(0u, 0u, 0u, 0u);
-          if (m < p.M) tv = __ldg(reinterpret_cast<const uint4*>(p.T + m * (long)lr_rank + 8 * v));
-          st_shared_v4(ts + (uint32_t)(row * t_pitch + 16 * v), tv);
+          const uint2 h = ld_shared_v2(l2b + (uint32_t)(i * 8));
+          st_shared_v4(l2s + (uint32_t)(i * 16), make_uint4(h.x << 16, h.x & 0xFFFF0000u, h.y << 16, h.y & 0xFFFF0000u));
         }
         named_barrier_sync(1, 16 * 32);
       }
@@ -911,8 +967,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sw[4], bv[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          sw[j] = __ldg(p.b_scale + n + j) * p.inv_group;
-          bv[j] = p.bias ? bf16_bits_to_float(__ldg(p.bias + n + j)) : 0.0f;
+          sw[j] = vec_sw[cs + j] * p.inv_group;
+          bv[j] = p.bias ? bf16_bits_to_float(vec_bias[cs + j]) : 0.0f;
         }
         for (int rb = row0; rb < BM; rb += 2 * step) {
           uint4 w[2][4];
@@ -921,7 +977,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 2; ++k) {
             const int row = rb + k * step;
             const long m = (long)tile_m(0) + row;
-            sa[k] = (row < BM && m < p.M) ? __ldg(p.a_scale + m) : 0.0f;
+            sa[k] = (row < BM && m < p.M) ? vec[row] : 0.0f;
             const uint32_t local = sbase + (uint32_t)(row * kPartPitch + c * 4);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
@@ -1084,11 +1140,11 @@ template <class Resident>
 bool choose_split(int tiles, int nkb, int rank, int sms, Resident&& resident, int& out) {
   out = 1;
   for (int s : {4, 2}) {
-    if (tiles * s > sms / 2 || nkb < 2 * s || rank * (256 / s) * 4 > kOutStageBytes) continue;
+    if (tiles * s > sms / 2 || nkb < 2 * s) continue;
     // the low-rank term runs on CUDA cores here (M N r fused multiply-adds,
     // ~0.13 us per unit of rank at M = 256, N = 3072): worth it only for a
     // small rank on a long K range
-    if (rank > 32 || (rank > 0 && nkb < 48)) continue;
+    if (rank > kSplitMaxRank || (rank > 0 && nkb < 48)) continue;
     int clusters = 0;
     if (!resident(s, clusters)) return false;
     if (clusters >= tiles) {
