@@ -53,8 +53,8 @@ def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
 # whitespace removed (so an edited comment keeps the figure, any code change
 # drops it to null).
 MEASURED_TRAFFIC = {
-    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "7763607990f1ad98", 11.890e6),
-    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "7763607990f1ad98", 20.498e6),
+    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "8b5fbab0aea008ae", 11.885e6),
+    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "8b5fbab0aea008ae", 20.501e6),
     ("rotate_quantize", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/quantize.cu", "003946100a4d56c2", 28.378e6),
 }
 
