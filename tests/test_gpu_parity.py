@@ -122,6 +122,8 @@ GEMM_CASES = [
     (1, 3072, 3072, 128, 0, True),      # split-K with a single token row
     (40, 8, 3072, 128, 0, False),       # split-K, one tile holding 8 of its 256 columns
     (256, 1024, 12288, 128, 32, True),  # split-K with the low-rank term in the reduction
+    (130, 520, 12288, 128, 16, True),   # the same with ragged M and N: zero-filled T rows and L2 columns
+    (3, 264, 6144, 128, 32, True),      # the same at three token rows
 ]
 
 
