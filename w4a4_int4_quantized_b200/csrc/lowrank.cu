@@ -30,7 +30,6 @@ namespace w4a4 {
 namespace {
 
 constexpr int BM = 128;        // rows of X per tile
-constexpr int BKL = 64;        // K per stage (128 bytes of bf16: one swizzle row)
 constexpr int NSTMAX = 8;      // TMA stages (as many as fit: 4 to 8)
 constexpr int kMaxSplit = 16;  // K split (cluster size): 16 needs the non-portable cluster size
 constexpr int kThreads = 128;
@@ -50,9 +49,12 @@ struct LrParams {
   int withhold;                 // self-test: the producer issues no operand load
 };
 
+// BKL: K per stage, 64 (one 128-byte swizzle atom of X per row) or 128 (two
+// atoms side by side: each row's 256 bytes are requested together, which
+// streams X faster where the ring still holds four stages, i.e. r <= 64).
 // MAXS: the largest split S this instantiation reduces (8 or 16; the
 // reduction loop is unrolled to it).
-template <int MAXS>
+template <int MAXS, int BKL>
 __global__ void __launch_bounds__(kThreads, 1)
     lowrank_down_kernel(const LrParams p, const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmL1) {
@@ -60,7 +62,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   const int rb = (p.r + 63) / 64;                       // 64-rank blocks of L1
-  const int kAB = BM * BKL * 2;                         // X stage: 16 KB
+  const int kAB = BM * BKL * 2;                         // X stage: BKL / 64 atoms of 16 KB
   const int kBB = rb * BKL * 128;                       // L1 stage: rb boxes of 64 K-rows x 128 bytes
   const int kStage = kAB + kBB;
   const int part_pitch = p.r * 4 + 16;                  // fp32 partial row pitch (padded)
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t st = sbase + (uint32_t)(s * kStage);
       mbar_arrive_expect_tx(&bar->full[s], (uint32_t)kStage);
-      tma_load_2d(st, &tmX, kb * BKL, m0, &bar->full[s]);
+      for (int a = 0; a < BKL / 64; ++a) tma_load_2d(st + a * (BM * 128), &tmX, kb * BKL + 64 * a, m0, &bar->full[s]);
       for (int b = 0; b < rb; ++b)
         tma_load_2d(st + kAB + b * (BKL * 128), &tmL1, b * 64, kb * BKL, &bar->full[s]);
       if (++s == NST) { s = 0; ph ^= 1u; }
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t st = sbase + (uint32_t)(s * kStage);
 #pragma unroll
       for (int ks = 0; ks < BKL / 16; ++ks)
-        mma_bf16_ss(tmem, smem_desc_kmajor_sw128(st + (uint32_t)(ks * 32)),
+        mma_bf16_ss(tmem, smem_desc_kmajor_sw128(st + (uint32_t)((ks >> 2) * (BM * 128) + (ks & 3) * 32)),
                     smem_desc_mnmajor_sw128(st + (uint32_t)(kAB + ks * 2048), BKL * 128, 1024), idesc,
                     (kb > kb0 || ks > 0) ? 1u : 0u);
       tc_commit(&bar->empty[s]);
@@ -214,6 +216,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 unsigned int* device_error_word();
 
+namespace {
+// the instantiation for a split S (clusters above 8 need the 16-wide
+// reduction) and a stage width of 128 (wide) or 64
+using LrKernel = void (*)(const LrParams, const CUtensorMap, const CUtensorMap);
+LrKernel kernel_for(int S, bool wide) {
+  if (wide) return S > 8 ? lowrank_down_kernel<kMaxSplit, 128> : lowrank_down_kernel<8, 128>;
+  return S > 8 ? lowrank_down_kernel<kMaxSplit, 64> : lowrank_down_kernel<8, 64>;
+}
+}  // namespace
+
 cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M, int K, int r, uint16_t* T,
                                    unsigned long long wait_ns, int withhold, cudaStream_t st) {
   unsigned int* err = device_error_word();
@@ -223,6 +235,9 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   if (e != cudaSuccess) return e;
   if ((e = device_sm_count(dev, &sms)) != cudaSuccess) return e;
   const int m_tiles = (M + BM - 1) / BM;
+  // 128-wide K stages where K allows and the ring keeps four of them
+  const bool wide = K % 128 == 0 && r <= 64;
+  const int BKL = wide ? 128 : 64;
   const int nkb = K / BKL;
   const int rb = (r + 63) / 64;
   const int stage = BM * BKL * 2 + rb * BKL * 128;
@@ -232,7 +247,8 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   const int smem = data + (int)sizeof(LrBarriers) + 1024;
   static DeviceFlags attr_set;
   if (!attr_set.done(dev)) {
-    for (auto k : {lowrank_down_kernel<8>, lowrank_down_kernel<kMaxSplit>}) {
+    for (auto k : {lowrank_down_kernel<8, 64>, lowrank_down_kernel<kMaxSplit, 64>, lowrank_down_kernel<8, 128>,
+                   lowrank_down_kernel<kMaxSplit, 128>}) {
       if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448)) != cudaSuccess ||
           (e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
         return e;
@@ -247,7 +263,7 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
     int64_t v[4];
   };
   static PlanCache<SKey, int, 32> split_cache;
-  SKey key = {{dev, m_tiles, nkb, smem}};
+  SKey key = {{dev, m_tiles, nkb, smem + ((int64_t)wide << 32)}};
   int S = 1;
   const bool ok = split_cache.get(key, S, [&](int& out) {
     out = 1;
@@ -265,8 +281,7 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
       qc.attrs = &qa;
       qc.numAttrs = 1;
       int max_clusters = 0;
-      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, sc > 8 ? lowrank_down_kernel<kMaxSplit> : lowrank_down_kernel<8>,
-                                               &qc)) != cudaSuccess)
+      if ((e = cudaOccupancyMaxActiveClusters(&max_clusters, kernel_for(sc, wide), &qc)) != cudaSuccess)
         return false;
       if (m_tiles <= max_clusters) out = sc;
     }
@@ -274,7 +289,7 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   });
   if (!ok) return e;
   CUtensorMap tX, tL1;
-  if (!make_tmap(&tX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)M, (uint64_t)K, BKL, BM,
+  if (!make_tmap(&tX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)M, (uint64_t)K, 64, BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tL1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L1, (uint64_t)K, (uint64_t)r, 64, BKL,
                  CU_TENSOR_MAP_SWIZZLE_128B))
@@ -294,8 +309,7 @@ cudaError_t launch_lowrank_down_ex(const uint16_t* X, const uint16_t* L1, int M,
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   LrParams prm{T, M, K, r, S, nst, err, wait_ns, withhold};
-  e = S > 8 ? cudaLaunchKernelEx(&cfg, lowrank_down_kernel<kMaxSplit>, prm, tX, tL1)
-            : cudaLaunchKernelEx(&cfg, lowrank_down_kernel<8>, prm, tX, tL1);
+  e = cudaLaunchKernelEx(&cfg, kernel_for(S, wide), prm, tX, tL1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
