@@ -7,7 +7,10 @@ activations (K1), then the INT4 GEMM with the fused dequant + bias epilogue
 (K2) -- the same two launches w4a4_linear makes.  Inputs are synthetic
 (seeded NumPy draws in the shape and value mix of the pages' workload) and
 resident in HBM; four input sets (about 272 MB) rotate so that no step finds
-its inputs in the 126 MB L2.
+its inputs in the 126 MB L2.  The K timed steps are captured once as a CUDA
+graph of layer calls and replayed (the launch pattern of a server running
+fixed-shape layers); the same K calls launched one by one from the host are
+reported beside it.
 
 Prints one JSON line (rank 0).  Metric: TOPS = 2 M N K / time.
 
@@ -700,18 +703,36 @@ def main():
             w4.w4a4_gemm(s["Xq"], s["xs"], s["Wq"], s["ws"], g, s["T"], s["L2"], s["bias"], Y=s["Y"],
                          stream=st)
 
-    def step(s):
+    def step(s, st=None):
         # one whole layer through the public call (its kernels: rotate +
         # quantize, the low-rank down-projection when r > 0, the GEMM)
+        st = stream if st is None else st
         if w4a8:
             w4.w4a8_linear(s["X"], s["Wq"], s["ws"], s["wz"], g, s["bias"], Y=s["Y"], workspace=s["work"],
-                           stream=stream)
+                           stream=st)
         else:
             w4.w4a4_linear(s["X"], s["Wq"], s["ws"], g, s["L1"], s["L2"], s["bias"], Y=s["Y"], workspace=s["work"],
-                           stream=stream)
+                           stream=st)
 
     for i in range(args.warmup):
         step(sets[i % len(sets)])
+    torch.cuda.synchronize()
+    # The K steps of the timed region are captured once as a CUDA graph (the
+    # way a server runs a fixed-shape layer: one replay launches every kernel
+    # of the K layers, with the same programmatic-launch overlap between
+    # them), so that the host's per-call cost is not timed as GPU work.  The
+    # same K calls launched one by one from the host are timed after it
+    # (`us_per_layer_direct`).
+    steps_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(steps_graph):
+        for i in range(args.steps):
+            step(sets[i % len(sets)], torch.cuda.current_stream())
+
+    def replay_steps():
+        with torch.cuda.stream(stream):
+            steps_graph.replay()
+
+    replay_steps()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -731,8 +752,7 @@ def main():
     wall0 = time.perf_counter()
     while args.soak_ms > 0 and (time.perf_counter() - wall0) * 1e3 < args.soak_ms:
         e_blk[0].record(stream)
-        for i in range(args.steps):
-            step(sets[i % len(sets)])
+        replay_steps()
         e_blk[1].record(stream)
         e_blk[1].synchronize()
         soak_ms.append(e_blk[0].elapsed_time(e_blk[1]) / args.steps)
@@ -742,8 +762,7 @@ def main():
         nb = torch.tensor([soak_blocks], device="cuda")
         dist.all_reduce(nb, op=dist.ReduceOp.MAX)
         for _ in range(int(nb.item()) - soak_blocks):
-            for i in range(args.steps):
-                step(sets[i % len(sets)])
+            replay_steps()
         torch.cuda.synchronize()
         dist.barrier()
     # timed region: K whole layers back to back (no events between kernels,
@@ -751,8 +770,7 @@ def main():
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_timed = time.perf_counter()
     e_start.record(stream)
-    for i in range(args.steps):
-        step(sets[i % len(sets)])
+    replay_steps()
     e_end.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t_timed
@@ -761,6 +779,14 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     total_ms = e_start.elapsed_time(e_end)
+    # the same K layers launched call by call from the host
+    e_start.record(stream)
+    for i in range(args.steps):
+        step(sets[i % len(sets)])
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    direct_ms = e_start.elapsed_time(e_end)
+    del steps_graph
 
     # per-kernel durations for the roofline: each kernel alone, back to back,
     # on the same rotating sets, replayed from a CUDA graph so that the host's
@@ -793,6 +819,7 @@ def main():
         raise SystemExit(f"device error word {err:#x}")
     from w4a4_int4_quantized_b200.shard import max_over_ranks
     total_ms = max_over_ranks(total_ms, device="cuda")
+    direct_ms = max_over_ranks(direct_ms, device="cuda")
     ops = 2.0 * M * N * K
     value = ops * args.steps * world / (total_ms * 1e-3) / 1e12
 
@@ -898,6 +925,7 @@ def main():
             "metric": _metric_name(args.variant, spec),
             "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "us_per_layer": total_ms / args.steps * 1e3,
+            "us_per_layer_direct": direct_ms / args.steps * 1e3,
             "frac_of_int8_nominal_peak": value / INT8_NOMINAL_TOPS,
             "layer_frac": {"of_int8_nominal": value / INT8_NOMINAL_TOPS,
                            "of_int8_measured": value / world / (2.0 * pk["bf16"]),
@@ -915,6 +943,9 @@ def main():
                        "lora_rank": args.lora,
                        "bias": spec.bias, "parallelism": f"replicas x{world} (token shards, no exchange)",
                        "l2": f"{args.sets} rotating input sets (> L2)",
+                       "launch": f"the K steps captured once as a CUDA graph of {'w4a8' if w4a8 else 'w4a4'}_linear "
+                                 "calls, replayed in the timed region (us_per_layer_direct: the same calls launched "
+                                 "one by one)",
                        "clock_soak_ms": args.soak_ms},
             "split_us": {"rotate_quantize": k1 * 1e3, "gemm": k2 * 1e3,
                          "note": "each kernel timed alone, back to back, replayed from a CUDA graph"},
