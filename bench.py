@@ -281,7 +281,7 @@ def run_mlp(args):
             step(sets[i % 2], fused)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             for i in range(n):
                 step(sets[i % 2], fused)
         graph.replay()
@@ -419,7 +419,7 @@ def run_block(args):
             fn()
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             for _ in range(n):
                 fn()
         graph.replay()
@@ -495,7 +495,7 @@ def run_sweep(args):
 
     def graph_of(fn, with_flush):
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             if with_flush:
                 flush.fill_(1)
             if fn is not None:
@@ -724,7 +724,7 @@ def main():
     # same K calls launched one by one from the host are timed after it
     # (`us_per_layer_direct`).
     steps_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(steps_graph):
+    with torch.cuda.graph(steps_graph, capture_error_mode="thread_local"):
         for i in range(args.steps):
             step(sets[i % len(sets)], torch.cuda.current_stream())
 
@@ -797,7 +797,7 @@ def main():
             fn(sets[i % len(sets)])
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             for i in range(n):
                 fn(sets[i % len(sets)], torch.cuda.current_stream())
         graph.replay()
