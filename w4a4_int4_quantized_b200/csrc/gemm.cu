@@ -934,10 +934,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // thread keeps one group of four columns (their scales and bias in
       // registers) and walks rows `step` apart, two rows' loads in flight.
       // With a low-rank branch (rank r = p.rank > 0) the slice's columns of
-      // L2 wait in the idle epilogue staging area as fp32 and its rows of T
-      // beside the partials, and each output adds sum_t T[m][t] L2[t][n]
-      // (fp32 fused multiply-adds, even and odd t in two chains) before the
-      // bias, like the persistent form's low-rank MMA does.
+      // L2 are widened to fp32 after the partials, its rows of T wait in the
+      // idle epilogue staging area, and each output adds sum_t T[m][t]
+      // L2[t][n] (fp32 fused multiply-adds, even and odd t in two chains)
+      // before the bias, like the persistent form's low-rank MMA does.
       const int S = prm.split;
       const int cw = BN / S;                             // columns in the slice
       const int per_row = cw / 4;                        // column groups in the slice
