@@ -215,7 +215,8 @@ def test_w4a8_weight_quant_special_rows():
 
 
 @pytest.mark.parametrize("M,N,K,g", [(64, 256, 256, 128), (200, 264, 384, 64), (2, 3072, 256, 128),
-                                     (257, 520, 3072, 0), (300, 768, 12288, 128)])
+                                     (257, 520, 3072, 0), (300, 768, 12288, 128),
+                                     (3, 264, 6144, 128)])   # split-K at three token rows, ragged N
 def test_w4a8_layer_parity(M, N, K, g):
     import torch
     d = _layer(M, N, K, g, 0, True, seed=M + N + K + 2)
@@ -272,7 +273,8 @@ def test_w4a4_layer_with_runtime_lora(M, N, K, g, r, rl, scale):
 
 
 @pytest.mark.parametrize("M,N,K,g,r", [(130, 520, 1280, 64, 32), (257, 768, 3072, 128, 0),
-                                     (256, 1024, 12288, 128, 32)])   # split-K, low-rank term in the reduction
+                                     (256, 1024, 12288, 128, 32),    # split-K, low-rank term in the reduction
+                                     (5, 264, 6144, 128, 16)])       # the same at five token rows, ragged N
 def test_w4a4_layer_with_fused_gelu(M, N, K, g, r):
     """GELU(tanh) fused into the epilogue: the same accumulators, GELU of the
     unrounded output within the layer tolerance, and the fused call equal to
