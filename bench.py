@@ -774,18 +774,19 @@ def main():
     e_end.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - t_timed
-    clocks.mark(wall0, t_timed + wall)
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
     total_ms = e_start.elapsed_time(e_end)
-    # the same K layers launched call by call from the host
+    # the same K layers launched call by call from the host, right after (the
+    # clock still at its loaded value)
     e_start.record(stream)
     for i in range(args.steps):
         step(sets[i % len(sets)])
     e_end.record(stream)
     torch.cuda.synchronize()
     direct_ms = e_start.elapsed_time(e_end)
+    clocks.mark(wall0, t_timed + wall)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
     del steps_graph
 
     # per-kernel durations for the roofline: each kernel alone, back to back,
