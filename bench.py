@@ -778,8 +778,10 @@ def main():
     # the same K layers launched call by call from the host, right after (the
     # clock still at its loaded value)
     e_start.record(stream)
+    t_host = time.perf_counter()
     for i in range(args.steps):
         step(sets[i % len(sets)])
+    host_us = (time.perf_counter() - t_host) / args.steps * 1e6   # host time to issue one call
     e_end.record(stream)
     torch.cuda.synchronize()
     direct_ms = e_start.elapsed_time(e_end)
@@ -926,7 +928,7 @@ def main():
             "metric": _metric_name(args.variant, spec),
             "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "us_per_layer": total_ms / args.steps * 1e3,
-            "us_per_layer_direct": direct_ms / args.steps * 1e3,
+            "us_per_layer_direct": direct_ms / args.steps * 1e3, "host_us_per_call": host_us,
             "frac_of_int8_nominal_peak": value / INT8_NOMINAL_TOPS,
             "layer_frac": {"of_int8_nominal": value / INT8_NOMINAL_TOPS,
                            "of_int8_measured": value / world / (2.0 * pk["bf16"]),
