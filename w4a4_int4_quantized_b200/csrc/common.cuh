@@ -222,6 +222,13 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool flag
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
+// A hint: bring the 2-D tile of `tmap` at (x, y) into L2 (no shared memory,
+// no barrier; later loads read memory as it then is).
+__device__ __forceinline__ void prefetch_tile_l2(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y)
+               : "memory");
+}
 
 // ---------------------------------------------------------------- proxies
 // Make this thread's generic-proxy shared-memory writes visible to the async

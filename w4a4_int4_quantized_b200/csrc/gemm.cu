@@ -310,6 +310,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
+      if constexpr (SPLIT != 0 || MODE == 2) {
+        // the weight tiles of this CTA's first k-blocks into L2 while the
+        // previous kernel finishes (a hint only: the loads after the
+        // dependency wait read the weights as that kernel left them).  Not in
+        // the persistent W4A4 forms, where the extra code costs spills.
+        if (my_tiles > 0) {
+          const int row_b = tile_n(0) + (int)rank * BNH;
+          for (int kb = 0; kb < min(PS, nk); ++kb) prefetch_tile_l2(&tmB, (kb0 + kb) * (PACKED ? BK / 2 : BK), row_b);
+        }
+      }
       prefetch_tmap(&tmY);
       if (LR) {
         prefetch_tmap(&tmT);
