@@ -56,8 +56,9 @@ def clock_adjusted_peak_tops(sm_mhz, sms: int = 148):
 # whitespace removed (so an edited comment keeps the figure, any code change
 # drops it to null).
 MEASURED_TRAFFIC = {
-    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "8b5fbab0aea008ae", 11.885e6),
-    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "8b5fbab0aea008ae", 20.501e6),
+    ("gemm", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "2109f93cdeed1d86", 11.892e6),
+    ("gemm", "m256_down"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "2109f93cdeed1d86", 20.503e6),
+    ("gemm_w4a8", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/gemm.cu", "2109f93cdeed1d86", 19.174e6),
     ("rotate_quantize", "attn_proj"): ("w4a4_int4_quantized_b200/csrc/quantize.cu", "003946100a4d56c2", 28.378e6),
 }
 
@@ -955,7 +956,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": k2_tops, "peak": int8_peak, "unit": "TOPS",
                          "frac": k2_tops / int8_peak,
                          "frac_clock_adjusted": (k2_tops / adj) if adj else None,
-                         "traffic": None if (w4a8 or r) else _traffic("gemm", spec.name),
+                         "traffic": None if r else _traffic("gemm_w4a8" if w4a8 else "gemm", spec.name),
                          "peak_note": f"int8 = 2 x {pk['source']} burst bf16 {pk['bf16']} TFLOP/s (kernel timed "
                                       f"alone); {2.0 * pk['bf16_sustained']:.0f} with the sustained figure"},
             "roofline_k1": {"bound": "hbm", "achieved": k1_bytes / (k1 * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
