@@ -118,6 +118,9 @@ w4a4_status w4a4_rotate_quantize_act(const void* X, int M, int K, int group, uin
  *   bias         bf16 [N] or NULL
  *   Y            out: bf16 [M, N]
  *   acc_debug    out: int32 [M, N] exact integer accumulators, or NULL
+ * Layers with too few 256 x 256 output tiles to occupy the GPU run a split-K
+ * form (w4a4_plan_gemm_split gives the decision); its int32 sums are exact,
+ * so Y is bit-identical to the persistent form's.
  */
 w4a4_status w4a4_gemm(const uint8_t* Xq, const float* x_scale, const uint8_t* Wq, const float* w_scale, int M,
                       int N, int K, int group, const void* T, const void* L2, int rank, const void* bias, void* Y,
