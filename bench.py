@@ -776,6 +776,8 @@ def main():
     torch.cuda.synchronize()
     wall = time.perf_counter() - t_timed
     total_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        dist.barrier()
     # the same K layers launched call by call from the host, right after (the
     # clock still at its loaded value)
     e_start.record(stream)
