@@ -47,3 +47,20 @@ def test_fewer_than_three_warmup_steps_are_refused():
                         "--warmup", "2"], cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert "warmup" in (r.stdout + r.stderr)
+
+
+def test_reference_arm_of_the_sweep_says_unavailable():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--sweep", "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["unavailable"]
+
+
+def test_reference_arm_of_the_w4a8_variant():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--variant", "w4a8", "--workload", "m256_down",
+                        "--steps", "1", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")][0]
+    assert d["impl"] == "reference" and d["value"] > 0 and "int8" in d["dtype"]
+    assert d["config"]["workload"] == "m256_down"
